@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Throughput of the LTX-2 joint audio-video block attention on B200.
+
+One step = the whole attention set of one DiT block (video self, audio self with
+the key-padding mask, v2a, a2v) over one batch of synthetic bf16 N(0,1) inputs,
+run back to back on one stream through the C ABI (libltxattn.so).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on a sample
+
+Prints one JSON line (rank 0).  ``value`` is the whole-job TFLOP/s (algorithmic
+FLOPs of all ranks / max-over-ranks device time); the timed region holds exactly
+K steps between barriers and device synchronisations, timed with CUDA events on
+the launching stream.  Multi-GPU runs are independent replicas (the attention of
+one block has no exchange step), hence weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s and µs/call per config; % of B200 dense-BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            lines = [ln.strip() for ln in f if ln.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                smax.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[6:10]):
+                if flag.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- oracle sample
+def oracle_sample(calls, fraction: float, seed: int):
+    """Time the fp64 oracle on ``fraction`` of every call's query rows (same mix of work)."""
+    import torch
+
+    from joint_audio_video_flash_b200 import synth
+    from oracle import oracle
+    flops = 0.0
+    secs = 0.0
+    rows_total = 0
+    g = torch.Generator().manual_seed(seed)
+    for c in calls:
+        q, k, v = synth.make_qkv(c.batch, c.q_len, c.kv_len, c.heads, c.head_dim, c.seed,
+                                 q_valid=c.q_valid, kv_valid=c.kv_valid_len)
+        n_rows = c.batch * c.q_valid * c.heads
+        take = max(1, int(round(n_rows * fraction)))
+        # real (unpadded) query rows only, sampled uniformly
+        pick = torch.randperm(n_rows, generator=g)[:take]
+        h = pick % c.heads
+        bi = pick // c.heads
+        i = bi % c.q_valid
+        b = bi // c.q_valid
+        rows = ((b * c.q_len + i) * c.heads + h).numpy()
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, c.scale, kv_valid_len=c.kv_valid_len, rows=rows)
+        secs += time.perf_counter() - t0
+        flops += 4.0 * take * c.kv_valid_len * c.head_dim
+        rows_total += take
+    return flops, secs, rows_total
+
+
+def cpu_baseline(calls, target_s: float, seed: int = 0):
+    from oracle import oracle
+    oracle.build()
+    total = sum(c.flops for c in calls)
+    # calibrate on a small sample, then size the measured sample to ~target_s
+    f0 = min(1.0, 2e9 / total)
+    fl, s, _ = oracle_sample(calls, f0, seed)
+    rate = fl / max(s, 1e-9)
+    frac = min(1.0, max(f0, target_s * rate / total))
+    fl, s, rows = oracle_sample(calls, frac, seed + 1)
+    return {"value": fl / s / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} query rows ({frac:.4%} of every call's real rows, same work mix), "
+                      f"{fl:.3e} FLOP in {s:.1f} s, fp64, OpenMP over rows"}
+
+
+# --------------------------------------------------------------------------- dist
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- main arms
+def run_reference(args):
+    from joint_audio_video_flash_b200 import workloads
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    desc, calls = workloads.configs()[args.workload]
+    from oracle import oracle
+    oracle.build()
+    total = sum(c.flops for c in calls)
+    per_step_s = max(2.0, args.reference_budget_s / (args.steps + args.warmup))
+    f0 = min(1.0, 1e9 / total)
+    fl, s, _ = oracle_sample(calls, f0, 0)
+    frac = min(1.0, max(f0, per_step_s * (fl / max(s, 1e-9)) / total))
+    for w in range(args.warmup):
+        oracle_sample(calls, f0, 100 + w)
+    flops = secs = 0.0
+    rows = 0
+    for st in range(args.steps):
+        a, b, r = oracle_sample(calls, frac, 1000 + st)
+        flops += a
+        secs += b
+        rows += r
+    value = flops / secs / 1e12
+    sample = (f"{rows} query rows over {args.steps} steps ({frac:.4%} of every call's real rows "
+              f"per step, same work mix), fp64 oracle, OpenMP over rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "description": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ltxattn(args):
+    import torch
+
+    from joint_audio_video_flash_b200 import build, ltxattn, synth, workloads
+
+    world, rank, local = dist_setup(args.gpus)
+    build.build()
+    ltxattn.create()
+    desc, calls = workloads.configs()[args.workload]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    host, dev_in, outs, splits = [], [], [], []
+    for c in calls:
+        q, k, v = synth.make_qkv(c.batch, c.q_len, c.kv_len, c.heads, c.head_dim, c.seed,
+                                 q_valid=c.q_valid, kv_valid=c.kv_valid_len)
+        host.append((q, k, v))
+        dev_in.append(tuple(t.to(dev) for t in (q, k, v)))
+        outs.append(torch.empty_like(dev_in[-1][0]))
+
+    def step(events=None):
+        for i, c in enumerate(calls):
+            dq, dk, dv = dev_in[i]
+            if events is not None:
+                events[i][0].record(stream)
+            _, used = ltxattn.forward(dq, dk, dv, outs[i], kv_valid_len=c.kv_valid_len,
+                                      scale=c.scale, return_splits=True)
+            if events is not None:
+                events[i][1].record(stream)
+            if len(splits) < len(calls):
+                splits.append(used)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    ltxattn.check()
+
+    per_call = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in calls] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    with ClockSampler(uuid) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for s in range(args.steps):
+            step(per_call[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ltxattn.check()
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    step_flops = sum(c.flops for c in calls)
+    value = step_flops * args.steps * world / (total_ms * 1e-3) / 1e12
+
+    call_us = []
+    for i, c in enumerate(calls):
+        ts = [per_call[s][i][0].elapsed_time(per_call[s][i][1]) * 1e3 for s in range(args.steps)]
+        call_us.append(ts)
+    launches_per_step = sum(1 if sp == 1 else 2 for sp in splits)
+
+    # ---- end to end through the public API with host buffers
+    pinned = [tuple(t.pin_memory() for t in trip) for trip in host]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for trip in pinned for t in trip)
+    d2h = sum(o.numel() * o.element_size() for o in host_out)
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for i, c in enumerate(calls):
+            dq, dk, dv = dev_in[i]
+            hq, hk, hv = pinned[i]
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            ltxattn.forward(dq, dk, dv, outs[i], kv_valid_len=c.kv_valid_len, scale=c.scale)
+            host_out[i].copy_(outs[i], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ltxattn.check()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    # dominant kernel: the video self-attention (tensor-core bound), timed inside the
+    # back-to-back step loop, so the sustained GEMM figure is its denominator
+    vi = max(range(len(calls)), key=lambda i: calls[i].flops)
+    v_us = statistics.mean(call_us[vi])
+    achieved = calls[vi].flops / (v_us * 1e-6) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": "fmha_fwd_sm100<128>",
+                "peak_source": f"{peak_src} bf16_tflops_sustained"}
+
+    per_call_out = {}
+    for i, c in enumerate(calls):
+        us = statistics.median(call_us[i])
+        tfl = c.flops / (us * 1e-6) / 1e12
+        gbs = c.bytes / (us * 1e-6) / 1e9
+        per_call_out[c.name] = {
+            "us_median": us, "us_p10": sorted(call_us[i])[max(0, int(0.1 * len(call_us[i])))],
+            "us_p90": sorted(call_us[i])[min(len(call_us[i]) - 1, int(0.9 * len(call_us[i])))],
+            "tflops": tfl, "frac_bf16_peak": tfl / float(peaks.get("bf16_tflops", 1590.0)),
+            "gbs": gbs, "frac_hbm": gbs / float(peaks.get("hbm_gbs", 6650.0)),
+            "shape": f"B{c.batch} Lq{c.q_len} Lkv{c.kv_len} valid{c.kv_valid_len} "
+                     f"H{c.heads} D{c.head_dim}",
+            "splits": splits[i]}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "description": desc,
+                   "l2": "inputs larger than L2 (video q/k/v alone exceed 126 MB per step)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "per_call": per_call_out,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(calls, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ltxattn", "reference"], default="ltxattn")
+    ap.add_argument("--workload", default="block768")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-budget-s", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ltxattn(args)
+
+
+if __name__ == "__main__":
+    main()

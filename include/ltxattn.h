@@ -1,0 +1,158 @@
+/*
+ * ltxattn.h -- C ABI of the B200 (sm_100a) attention library for the LTX-2 joint
+ * audio-video diffusion transformer block.
+ *
+ * What is computed.  For every batch element b, head h and query row i:
+ *     s_j = scale * sum_d q[b,i,h,d] * k[b,j,h,d]          for keys j < kv_valid_len
+ *     o[b,i,h,:] = sum_j exp(s_j - max s) v[b,j,h,:] / sum_j exp(s_j - max s)
+ * which covers the four attentions of a block: video self-attention over the
+ * video latent tokens, audio self-attention over the (padded) audio tokens, v2a
+ * (audio queries over video keys/values) and a2v (video queries over audio
+ * keys/values), as described in "LTX-2: replicate audio stream across Ulysses
+ * ranks by default" (TensorRT-LLM pull request 16228), Description.  Keys at
+ * index >= kv_valid_len are masked out: the audio stream is zero-padded before
+ * attention (same Description), and the padded keys must not contribute.
+ *
+ * Layout.  All four tensors are bf16, contiguous, BSHD:
+ *     q, out : [batch, q_len,  heads, head_dim]
+ *     k, v   : [batch, kv_len, heads, head_dim]
+ * element (b, s, h, d) at ((b*len + s)*heads + h)*head_dim + d.  Queries and
+ * keys share `heads` and `head_dim`.
+ *
+ * Precision.  bf16 inputs, fp32 accumulation (tensor-core MMAs into tensor
+ * memory), fp32 softmax statistics, probabilities rounded to bf16 before the
+ * P*V product, output rounded to bf16 (round to nearest even).
+ *
+ * Ownership.  The caller owns q, k, v and out (device memory) and the stream;
+ * the library never frees them.  The library owns a per-device context (device
+ * status word, tensor-map encoder) and per-stream workspace for key-range
+ * partials, allocated in stream order on first need and released by
+ * ltxattn_destroy.
+ *
+ * Threading.  Calls on one device may come from any host thread.  Calls on the
+ * same stream are ordered by the stream; calls on different streams use separate
+ * workspaces.
+ *
+ * Errors.  Every entry point returns an ltxattn_status.  Argument checks run on
+ * the host, before any CUDA call and before anything is enqueued, so a rejected
+ * call has no effect.  Compute calls are asynchronous on `stream` and never
+ * synchronise.  A kernel that finds its pipeline stalled past the library's
+ * wait limit records LTXATTN_ERR_DEVICE_TIMEOUT in the device status word and
+ * returns instead of hanging; ltxattn_check reads (and clears) that word.
+ */
+#ifndef LTXATTN_H_
+#define LTXATTN_H_
+
+#if defined(__GNUC__)
+#define LTXATTN_API __attribute__((visibility("default")))
+#else
+#define LTXATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* ltxattn_stream_t;
+
+typedef enum {
+  LTXATTN_OK = 0,
+  LTXATTN_ERR_INVALID_ARG = 1,     /* null pointer, bad size, kv_valid_len outside [1, kv_len],
+                                      non-finite or non-positive scale, out aliasing an input */
+  LTXATTN_ERR_UNSUPPORTED = 2,     /* head_dim not in {64, 128}, or a size beyond the limits */
+  LTXATTN_ERR_MISALIGNED = 3,      /* a tensor base address not 16-byte aligned */
+  LTXATTN_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
+  LTXATTN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel hit its wait limit (see ltxattn_check) */
+  LTXATTN_ERR_NOT_INITIALIZED = 6  /* no context on the current device: call ltxattn_create */
+} ltxattn_status;
+
+/* Largest sizes accepted (larger values give LTXATTN_ERR_UNSUPPORTED). */
+#define LTXATTN_MAX_LEN (1 << 24)   /* q_len, kv_len */
+#define LTXATTN_MAX_HEADS 1024
+#define LTXATTN_MAX_BATCH 1024
+
+/*
+ * Creates the context for the CUDA device current on the calling thread:
+ * device properties, a zeroed device status word and the kernels' shared-memory
+ * limits.  Idempotent: a second call on the same device returns LTXATTN_OK.
+ * Errors: LTXATTN_ERR_CUDA (no device, allocation or attribute failure).
+ */
+LTXATTN_API int ltxattn_create(void);
+
+/*
+ * Attention forward on the current device, enqueued on `stream`.
+ *   q, k, v     device pointers, bf16 BSHD as above, 16-byte aligned.
+ *   out         device pointer, bf16 BSHD [batch, q_len, heads, head_dim],
+ *               16-byte aligned, not overlapping q, k or v.
+ *   q_len       query rows, 1 .. LTXATTN_MAX_LEN.  Query rows beyond the real
+ *               tokens (padding) are computed like any other row.
+ *   kv_len      key/value rows, 1 .. LTXATTN_MAX_LEN.
+ *   kv_valid_len  keys [0, kv_valid_len) take part; 1 <= kv_valid_len <= kv_len.
+ *               Keys are staged in whole 128-row tiles, so the value rows of
+ *               the last, partially valid tile beyond kv_valid_len are read
+ *               (with zero weight): they must be finite (zero padding is).
+ *   batch, heads  1 .. LTXATTN_MAX_BATCH, 1 .. LTXATTN_MAX_HEADS.
+ *   head_dim    64 or 128.
+ *   scale       softmax scale, finite and > 0 (typically 1/sqrt(head_dim)).
+ *   stream      CUDA stream (NULL = default stream).
+ * Returns LTXATTN_OK once the work is enqueued, or the first failing check:
+ * INVALID_ARG, UNSUPPORTED, MISALIGNED (all before any CUDA call),
+ * NOT_INITIALIZED, CUDA (launch or workspace failure).
+ */
+LTXATTN_API int ltxattn_forward(const void* q, const void* k, const void* v, void* out, int q_len, int kv_len,
+                    int kv_valid_len, int batch, int heads, int head_dim, float scale,
+                    ltxattn_stream_t stream);
+
+/*
+ * ltxattn_forward with an explicit plan.  num_splits = 0 lets the library choose
+ * (as ltxattn_forward does); num_splits >= 1 asks for that many key-range parts
+ * merged through their softmax statistics (clamped to the number of 128-key
+ * tiles; 1 = no split).  If splits_used is not NULL it receives the number of
+ * parts actually launched.  Same errors as ltxattn_forward, plus INVALID_ARG for
+ * num_splits < 0.
+ */
+LTXATTN_API int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, int q_len,
+                       int kv_len, int kv_valid_len, int batch, int heads, int head_dim,
+                       float scale, int num_splits, int* splits_used, ltxattn_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  Returns LTXATTN_ERR_DEVICE_TIMEOUT if a kernel recorded a
+ * stalled wait since the last check, LTXATTN_ERR_CUDA if the synchronisation
+ * failed, LTXATTN_ERR_NOT_INITIALIZED without a context, else LTXATTN_OK.
+ */
+LTXATTN_API int ltxattn_check(ltxattn_stream_t stream);
+
+/*
+ * Synchronises the current device, checks the status word (as ltxattn_check)
+ * and frees the context and all workspaces of the current device.  Returns the
+ * status check's result; LTXATTN_ERR_NOT_INITIALIZED without a context.
+ */
+LTXATTN_API int ltxattn_destroy(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+LTXATTN_API const char* ltxattn_status_string(int status);
+
+/*
+ * Self-test of the failure path: launches one CTA that waits on a barrier no
+ * one arrives at, with a wait limit of `timeout_ns` nanoseconds (1e3 .. 1e10),
+ * then synchronises `stream` and returns what ltxattn_check returns
+ * (LTXATTN_ERR_DEVICE_TIMEOUT when the bounded wait works).  The status word is
+ * cleared afterwards, so later calls are unaffected.
+ */
+LTXATTN_API int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltxattn_stream_t stream);
+
+/*
+ * Number of entry points above, and their names, for loaders that check the
+ * exported symbols.
+ */
+LTXATTN_API int ltxattn_num_entry_points(void);
+LTXATTN_API const char* ltxattn_entry_point_name(int i);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LTXATTN_H_ */

@@ -1,0 +1,396 @@
+// fmha_fwd.cuh -- flash-style softmax attention forward for sm_100a.
+//
+// Computes O = softmax(scale * Q K^T + M) V per (batch, head) for the four
+// attentions of an LTX-2 joint audio-video DiT block (video self, audio self,
+// v2a = audio queries over video keys/values, a2v = video queries over audio
+// keys/values; "LTX-2: replicate audio stream across Ulysses ranks by default",
+// Description).  M is -inf on keys >= kv_valid (the zero-padded audio tail, same
+// Description) and 0 elsewhere.  Tensors are bf16 BSHD: element (b, s, h, d) at
+// ((b*len + s)*heads + h)*D + d.
+//
+// One CTA owns one 128-row query tile of one (batch, head) and streams 128-key
+// tiles of K and V through shared memory:
+//   warp 0      TMA producer: Q once, then K_j and V_j into 2-stage rings.
+//   warp 1      MMA issuer: S_j = Q K_j^T (SS, bf16 -> fp32 in TMEM, S double
+//               buffered) and O += P_j V_j (A = P read from TMEM, B = V from smem).
+//   warps 2-5   softmax: one query row per thread (TMEM lane = row); row max with a
+//               lazy rescale of O (only when the running max grows by > 2^8), exp2
+//               on the MUFU, fp32 row sums, P written back over S as packed bf16;
+//               then the epilogue.
+// TMEM columns: S buffer 0 at [0,128), S buffer 1 at [128,256), O at [256,256+D).
+//
+// In split mode (short query side, long key side: v2a) the CTA covers one range
+// of key tiles and writes its normalised fp32 partial output and its base-2
+// log-sum-exp; combine.cuh merges the parts through those statistics (the merge of
+// per-rank softmax statistics in "feat(ltx2): tile-parallel video VAE and the
+// two-stage pipeline", commit "Onboard Lightricks LTX-2.5").
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace ltx {
+
+constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
+constexpr int kBlockN = 128;  // keys per tile
+constexpr int kFwdThreads = 192;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
+constexpr int kMinSmemFor1Cta = 120 * 1024;  // forces one CTA per SM (TMEM holds 512 columns)
+
+struct FwdParams {
+  int q_len;
+  int kv_len;
+  int kv_valid;
+  int heads;
+  int batch;
+  int n_q_tiles;        // ceil(q_len / 128)
+  int n_kv_tiles;       // ceil(kv_valid / 128)
+  int num_splits;       // key-range parts (1 = direct bf16 output)
+  int tiles_per_split;  // key tiles per part
+  float scale_log2;     // scale * log2(e)
+  float* o_part;        // split: [splits][batch][heads][n_q_tiles*128][D] fp32
+  float* lse_part;      // split: [splits][batch][heads][n_q_tiles*128] base-2 LSE
+  int* status;          // device status word
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kBoxes = D / 64;             // 128-byte (64 x bf16) column boxes per row
+  static constexpr int kBoxBytes = kBlockM * 128;   // one 128-row x 64-column box
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kStages = (D == 64) ? 3 : 2;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  // barriers
+  static constexpr int bQ = 0;
+  static constexpr int bKF = 1;
+  static constexpr int bKE = bKF + kStages;
+  static constexpr int bVF = bKE + kStages;
+  static constexpr int bVE = bVF + kStages;
+  static constexpr int bSF = bVE + kStages;  // 2
+  static constexpr int bPF = bSF + 2;        // 2
+  static constexpr int bOD = bPF + 2;        // O updated by a PV
+  static constexpr int bOF = bOD + 1;        // final PV done
+  static constexpr int bDrain = bOF + 1;     // abort-path drain
+  static constexpr int kNumBars = bDrain + 1;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kUsed = kAbort + 4;
+  static constexpr int kAlloc = ((kUsed + 1024 + 1023) / 1024) * 1024 > kMinSmemFor1Cta
+                                    ? ((kUsed + 1024 + 1023) / 1024) * 1024
+                                    : kMinSmemFor1Cta;
+  static constexpr int kColO = 256;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// Bounded wait that ignores the abort flag (used to drain copies / MMAs on the
+// abort path before the CTA releases shared and tensor memory).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
+                                                unsigned long long timeout_ns) {
+  const unsigned long long t0 = global_timer_ns();
+  const unsigned long long max_spins = timeout_ns / 4 + 1024;
+  unsigned long long spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns || ++spins > max_spins) return false;
+  }
+  return true;
+}
+
+template <int D, bool kSplit>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const FwdParams p) {
+  using L = FwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qt = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = kSplit ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z;
+  const int split = kSplit ? (int)blockIdx.z % p.num_splits : 0;
+  const int kv_begin = split * p.tiles_per_split;
+  const int kv_end = min(kv_begin + p.tiles_per_split, p.n_kv_tiles);
+  const int n = kv_end - kv_begin;  // >= 1 by construction on the host
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::bQ), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::bKF + s), 1);
+      mbar_init(bar(L::bKE + s), 1);
+      mbar_init(bar(L::bVF + s), 1);
+      mbar_init(bar(L::bVE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::bSF + s), 1);
+      mbar_init(bar(L::bPF + s), kBlockM);
+    }
+    mbar_init(bar(L::bOD), 1);
+    mbar_init(bar(L::bOF), 1);
+    mbar_init(bar(L::bDrain), 1);
+    // a CTA that starts after another one failed does no work
+    *abort_flag = (*reinterpret_cast<volatile int*>(p.status) != kDevOk) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::kTmemSlot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && !*abort_flag) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(L::bQ), L::kTileBytes);
+      for (int bx = 0; bx < L::kBoxes; ++bx)
+        tma_load_4d(sbase + L::kQ + bx * L::kBoxBytes, &tm_q, bar(L::bQ), bx * 64, h,
+                    qt * kBlockM, b);
+      int last_k[L::kStages], last_v[L::kStages];
+      for (int s = 0; s < L::kStages; ++s) last_k[s] = last_v[s] = -1;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % L::kStages;
+        const uint32_t ph = (uint32_t)(j / L::kStages) & 1u;
+        const int kv0 = (kv_begin + j) * kBlockN;
+        ok = mbar_wait(bar(L::bKE + st), ph ^ 1u, ctl);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(L::bKF + st), L::kTileBytes);
+        for (int bx = 0; bx < L::kBoxes; ++bx)
+          tma_load_4d(sbase + L::kK + st * L::kTileBytes + bx * L::kBoxBytes, &tm_k,
+                      bar(L::bKF + st), bx * 64, h, kv0, b);
+        last_k[st] = j;
+        ok = mbar_wait(bar(L::bVE + st), ph ^ 1u, ctl);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(L::bVF + st), L::kTileBytes);
+        for (int bx = 0; bx < L::kBoxes; ++bx)
+          tma_load_4d(sbase + L::kV + st * L::kTileBytes + bx * L::kBoxBytes, &tm_v,
+                      bar(L::bVF + st), bx * 64, h, kv0, b);
+        last_v[st] = j;
+      }
+      if (!ok) {
+        // let every copy this thread started land before shared memory is released
+        for (int s = 0; s < L::kStages; ++s) {
+          if (last_k[s] >= 0)
+            mbar_wait_drain(bar(L::bKF + s), (uint32_t)(last_k[s] / L::kStages) & 1u, p.timeout_ns);
+          if (last_v[s] >= 0)
+            mbar_wait_drain(bar(L::bVF + s), (uint32_t)(last_v[s] / L::kStages) & 1u, p.timeout_ns);
+        }
+        mbar_wait_drain(bar(L::bQ), 0, p.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !*abort_flag) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
+      bool ok = mbar_wait(bar(L::bQ), 0, ctl);
+      bool issued = false;
+      auto pv = [&](int t) -> bool {
+        const int sb = t & 1;
+        if (!mbar_wait(bar(L::bPF + sb), (uint32_t)(t >> 1) & 1u, ctl)) return false;
+        const int st = t % L::kStages;
+        if (!mbar_wait(bar(L::bVF + st), (uint32_t)(t / L::kStages) & 1u, ctl)) return false;
+        tc_fence_after();
+        const uint32_t v_base = sbase + L::kV + st * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          // B = V tile, N = D (MN-major: d contiguous), K = 16 keys starting at kk*16
+          const uint64_t bdesc = smem_desc_sw128(v_base + kk * 16 * 128, L::kBoxBytes, 1024);
+          umma_ts(tmem + L::kColO, tmem + sb * 128 + kk * 8, bdesc, idesc_pv,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar(L::bVE + st));
+        umma_commit(bar(L::bOD));
+        return true;
+      };
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j % L::kStages;
+        ok = mbar_wait(bar(L::bKF + st), (uint32_t)(j / L::kStages) & 1u, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        const int sb = j & 1;
+        const uint32_t k_base = sbase + L::kK + st * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          const uint64_t adesc = smem_desc_sw128(sbase + L::kQ + off, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
+          umma_ss(tmem + sb * 128, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        umma_commit(bar(L::bSF + sb));
+        umma_commit(bar(L::bKE + st));
+        if (j >= 1) ok = pv(j - 1);
+      }
+      if (ok) ok = pv(n - 1);
+      if (ok) {
+        umma_commit(bar(L::bOF));
+      } else if (issued) {
+        // all MMAs this thread issued must finish before TMEM is released
+        umma_commit(bar(L::bDrain));
+        mbar_wait_drain(bar(L::bDrain), 0, p.timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wq = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = wq * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY;
+    float l_run = 0.0f;
+    bool ok = !*abort_flag;
+    for (int j = 0; j < n && ok; ++j) {
+      const int sb = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(j >> 1) & 1u, ctl));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kBlockN];
+#pragma unroll
+      for (int c = 0; c < kBlockN / 32; ++c)
+        tmem_ld32(trow + sb * 128 + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+      tmem_ld_wait();
+      const int kv0 = (kv_begin + j) * kBlockN;
+      if (kv0 + kBlockN > p.kv_valid) {
+        const int lim = p.kv_valid - kv0;
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+      mx *= sl2;
+      if (j == 0) {
+        m_run = mx;
+      } else if (__any_sync(0xffffffffu, mx > m_run + kRescaleThreshold)) {
+        // Warp-uniform branch (tcgen05.ld/st are warp-collective): every lane of the
+        // warp moves to its own new max; lanes whose max did not grow scale by 1.
+        // O must hold the PV of tile j-1 before it is rescaled.
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOD), (uint32_t)(j - 1) & 1u, ctl));
+        if (!ok) break;
+        tc_fence_after();
+        mx = fmaxf(mx, m_run);
+        const float f = ex2(m_run - mx);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(trow + L::kColO + c * 32, o);
+          tmem_ld_wait();
+          uint32_t u[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(o[x] * f);
+          tmem_st32(trow + L::kColO + c * 32, u);
+        }
+        tmem_st_wait();
+        l_run *= f;
+        m_run = mx;
+      }
+      const float neg_m = -m_run;
+      float sum = 0.0f;
+#pragma unroll
+      for (int c = 0; c < kBlockN / 64; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const float p0 = ex2(fmaf(s[c * 64 + 2 * x], sl2, neg_m));
+          const float p1 = ex2(fmaf(s[c * 64 + 2 * x + 1], sl2, neg_m));
+          sum += p0 + p1;
+          pk[x] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(trow + sb * 128 + c * 32, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::bPF + sb));
+      l_run += sum;
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOF), 0, ctl));
+    // every softmax thread gets here (all waits are bounded); agree on one outcome so
+    // that the epilogue's named barrier is reached by all 128 threads or by none
+    ok = named_bar_and(1, kBlockM, ok && !*abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      if constexpr (!kSplit) {
+        // normalise, round to bf16, stage in the (now idle) Q tile with the
+        // 128-byte swizzle the output tensor map expects, then one TMA store
+        uint8_t* stage = smem + L::kQ;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(trow + L::kColO + c * 32, o);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) w[x] = pack_bf16x2(o[2 * x] * inv_l, o[2 * x + 1] * inv_l);
+          const int bx = c >> 1;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
+            uint4* dst = reinterpret_cast<uint4*>(stage + bx * L::kBoxBytes + row * 128 +
+                                                  ((chunk ^ (row & 7)) << 4));
+            *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, kBlockM);
+        if (threadIdx.x == 64) {
+          for (int bx = 0; bx < L::kBoxes; ++bx)
+            tma_store_4d(&tm_o, sbase + L::kQ + bx * L::kBoxBytes, bx * 64, h, qt * kBlockM, b);
+          tma_store_commit();
+          tma_store_wait_read0();
+        }
+      } else {
+        const int rows_pad = p.n_q_tiles * kBlockM;
+        const int grow = qt * kBlockM + row;
+        const bool live = grow < p.q_len;  // padded tail rows of the last tile are not stored
+        const size_t prow =
+            (((size_t)split * p.batch + b) * p.heads + h) * (size_t)rows_pad + (size_t)grow;
+        float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          __syncwarp();
+          tmem_ld32(trow + L::kColO + c * 32, o);  // warp-collective: every lane loads
+          tmem_ld_wait();
+          if (live) {
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              dst[c * 8 + x] = make_float4(o[4 * x] * inv_l, o[4 * x + 1] * inv_l,
+                                           o[4 * x + 2] * inv_l, o[4 * x + 3] * inv_l);
+          }
+        }
+        if (live) p.lse_part[prow] = m_run + __log2f(l_run);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace ltx

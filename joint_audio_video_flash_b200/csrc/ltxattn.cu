@@ -1,0 +1,378 @@
+// ltxattn.cu -- host side of the C ABI declared in include/ltxattn.h: argument
+// validation, per-device context, TMA tensor maps, key-range split planning,
+// workspace and kernel launches.  No CPU compute path exists: every step of the
+// attention runs in the kernels of fmha_fwd.cuh and combine.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <map>
+#include <mutex>
+
+#include "../../include/ltxattn.h"
+#include "combine.cuh"
+#include "fmha_fwd.cuh"
+
+namespace {
+
+using ltx::FwdParams;
+using ltx::FwdSmem;
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+struct Context {
+  int device = -1;
+  int num_sms = 0;
+  int* d_status = nullptr;
+  EncodeTiledFn encode = nullptr;
+  std::map<cudaStream_t, Workspace> workspaces;
+};
+
+std::mutex g_mu;
+std::map<int, Context*> g_ctx;
+
+const char* const kEntryPoints[] = {
+    "ltxattn_create",        "ltxattn_forward",          "ltxattn_forward_ex",
+    "ltxattn_check",         "ltxattn_destroy",          "ltxattn_status_string",
+    "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
+};
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// All checks that need no CUDA call, in the order the header documents.
+int validate(const void* q, const void* k, const void* v, void* out, int q_len, int kv_len,
+             int kv_valid_len, int batch, int heads, int head_dim, float scale) {
+  if (!q || !k || !v || !out) return LTXATTN_ERR_INVALID_ARG;
+  if (q_len < 1 || kv_len < 1 || batch < 1 || heads < 1) return LTXATTN_ERR_INVALID_ARG;
+  if (kv_valid_len < 1 || kv_valid_len > kv_len) return LTXATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return LTXATTN_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LTXATTN_ERR_UNSUPPORTED;
+  if (q_len > LTXATTN_MAX_LEN || kv_len > LTXATTN_MAX_LEN || heads > LTXATTN_MAX_HEADS ||
+      batch > LTXATTN_MAX_BATCH)
+    return LTXATTN_ERR_UNSUPPORTED;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+  if (mis & 15u) return LTXATTN_ERR_MISALIGNED;
+  const size_t row = (size_t)heads * head_dim * 2;
+  const size_t nq = (size_t)batch * q_len * row, nkv = (size_t)batch * kv_len * row;
+  if (overlaps(out, nq, q, nq) || overlaps(out, nq, k, nkv) || overlaps(out, nq, v, nkv))
+    return LTXATTN_ERR_INVALID_ARG;
+  return LTXATTN_OK;
+}
+
+// BSHD bf16 tensor [batch, len, heads, head_dim] seen as a 4-D TMA tensor
+// (d, h, s, b) with a 64-column x 128-row box and the 128-byte swizzle.
+bool encode_bshd(const Context& c, CUtensorMap* map, const void* base, int len, int batch,
+                 int heads, int head_dim) {
+  const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)heads, (cuuint64_t)len,
+                              (cuuint64_t)batch};
+  const cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)heads * head_dim * 2,
+                                 (cuuint64_t)len * heads * head_dim * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)ltx::kBlockM, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = c.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Key-range parts: enough (b, h, q-tile) x part CTAs to fill the SMs without
+// over-splitting.  Cost model: waves x (tiles per part + fixed per-CTA overhead).
+int plan_splits(int units, int n_kv_tiles, int num_sms) {
+  if (n_kv_tiles < 4 || units >= num_sms) return 1;
+  const int kOverheadTiles = 2;
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= std::min(n_kv_tiles, 64); ++s) {
+    const long long waves = ((long long)units * s + num_sms - 1) / num_sms;
+    const long long cost = waves * ((n_kv_tiles + s - 1) / s + kOverheadTiles);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+Context* current_context(int* err) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    *err = LTXATTN_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_ctx.find(dev);
+  if (it == g_ctx.end()) {
+    *err = LTXATTN_ERR_NOT_INITIALIZED;
+    return nullptr;
+  }
+  *err = LTXATTN_OK;
+  return it->second;
+}
+
+template <int D, bool kSplit>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
+  dim3 grid(p.n_q_tiles, p.heads, p.batch * p.num_splits);
+  ltx::fmha_fwd_sm100<D, kSplit><<<grid, ltx::kFwdThreads, FwdSmem<D>::kAlloc, stream>>>(
+      tq, tk, tv, to, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_combine(const FwdParams& p, void* out, cudaStream_t stream) {
+  const long long total = (long long)p.batch * p.q_len * p.heads * (D / 4);
+  const long long blocks = (total + ltx::kCombineThreads - 1) / ltx::kCombineThreads;
+  ltx::combine_splits<D><<<(unsigned)blocks, ltx::kCombineThreads, 0, stream>>>(
+      p.o_part, p.lse_part, reinterpret_cast<__nv_bfloat16*>(out), p.num_splits, p.batch, p.heads,
+      p.q_len, p.n_q_tiles * ltx::kBlockM);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t set_smem_limits() {
+  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_sm100<D, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FwdSmem<D>::kAlloc);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ltx::fmha_fwd_sm100<D, true>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<D>::kAlloc);
+}
+
+__global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ltx::mbar_init(ltx::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ltx::fence_mbar_init();
+  }
+  __syncthreads();
+  const ltx::WaitCtl ctl{&abort_flag, status, timeout_ns};
+  // nothing ever arrives on the barrier, so phase 0 never completes
+  if (threadIdx.x == 0) ltx::mbar_wait(ltx::smem_u32(&bar), 0, ctl);
+  __syncthreads();
+}
+
+int read_and_clear_status(Context* c, cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  int h = 0;
+  if (cudaMemcpy(&h, c->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LTXATTN_ERR_CUDA;
+  if (h != ltx::kDevOk) {
+    if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return LTXATTN_ERR_CUDA;
+    return LTXATTN_ERR_DEVICE_TIMEOUT;
+  }
+  return LTXATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ltxattn_create(void) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_ctx.count(dev)) return LTXATTN_OK;
+  Context* c = new Context();
+  c->device = dev;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  bool ok = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) ==
+                cudaSuccess &&
+            cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && fn != nullptr;
+  if (ok) {
+    c->encode = reinterpret_cast<EncodeTiledFn>(fn);
+    ok = cudaMalloc(&c->d_status, sizeof(int)) == cudaSuccess &&
+         cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
+         set_smem_limits<64>() == cudaSuccess && set_smem_limits<128>() == cudaSuccess &&
+         cudaDeviceSynchronize() == cudaSuccess;
+  }
+  if (!ok) {
+    cudaGetLastError();
+    if (c->d_status) cudaFree(c->d_status);
+    delete c;
+    return LTXATTN_ERR_CUDA;
+  }
+  g_ctx[dev] = c;
+  return LTXATTN_OK;
+}
+
+int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, int q_len,
+                       int kv_len, int kv_valid_len, int batch, int heads, int head_dim,
+                       float scale, int num_splits, int* splits_used, ltxattn_stream_t stream_) {
+  int st = validate(q, k, v, out, q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale);
+  if (st != LTXATTN_OK) return st;
+  if (num_splits < 0) return LTXATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  Context* c = current_context(&st);
+  if (!c) return st;
+
+  FwdParams p{};
+  p.q_len = q_len;
+  p.kv_len = kv_len;
+  p.kv_valid = kv_valid_len;
+  p.heads = heads;
+  p.batch = batch;
+  p.n_q_tiles = (q_len + ltx::kBlockM - 1) / ltx::kBlockM;
+  p.n_kv_tiles = (kv_valid_len + ltx::kBlockN - 1) / ltx::kBlockN;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = c->d_status;
+  p.timeout_ns = kDefaultTimeoutNs;
+
+  const int units = p.n_q_tiles * heads * batch;
+  int splits = num_splits > 0 ? std::min(num_splits, p.n_kv_tiles)
+                              : plan_splits(units, p.n_kv_tiles, c->num_sms);
+  p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
+  splits = (p.n_kv_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty part
+  if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
+  p.num_splits = splits;
+  if (splits_used) *splits_used = splits;
+
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bshd(*c, &tq, q, q_len, batch, heads, head_dim) ||
+      !encode_bshd(*c, &tk, k, kv_len, batch, heads, head_dim) ||
+      !encode_bshd(*c, &tv, v, kv_len, batch, heads, head_dim) ||
+      !encode_bshd(*c, &to, out, q_len, batch, heads, head_dim))
+    return LTXATTN_ERR_CUDA;
+
+  if (splits > 1) {
+    const size_t rows = (size_t)splits * batch * heads * (size_t)p.n_q_tiles * ltx::kBlockM;
+    const size_t o_bytes = rows * head_dim * sizeof(float);
+    const size_t need = o_bytes + rows * sizeof(float);
+    Workspace* ws;
+    {
+      std::lock_guard<std::mutex> lk(g_mu);
+      ws = &c->workspaces[stream];
+    }
+    if (ws->bytes < need) {
+      if (ws->ptr && cudaFreeAsync(ws->ptr, stream) != cudaSuccess) return LTXATTN_ERR_CUDA;
+      ws->ptr = nullptr;
+      ws->bytes = 0;
+      if (cudaMallocAsync(&ws->ptr, need, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LTXATTN_ERR_CUDA;
+      }
+      ws->bytes = need;
+    }
+    p.o_part = reinterpret_cast<float*>(ws->ptr);
+    p.lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws->ptr) + o_bytes);
+  }
+
+  cudaError_t e;
+  if (head_dim == 64) {
+    e = splits > 1 ? launch_fwd<64, true>(tq, tk, tv, to, p, stream)
+                   : launch_fwd<64, false>(tq, tk, tv, to, p, stream);
+    if (e == cudaSuccess && splits > 1) e = launch_combine<64>(p, out, stream);
+  } else {
+    e = splits > 1 ? launch_fwd<128, true>(tq, tk, tv, to, p, stream)
+                   : launch_fwd<128, false>(tq, tk, tv, to, p, stream);
+    if (e == cudaSuccess && splits > 1) e = launch_combine<128>(p, out, stream);
+  }
+  return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
+int ltxattn_forward(const void* q, const void* k, const void* v, void* out, int q_len, int kv_len,
+                    int kv_valid_len, int batch, int heads, int head_dim, float scale,
+                    ltxattn_stream_t stream) {
+  return ltxattn_forward_ex(q, k, v, out, q_len, kv_len, kv_valid_len, batch, heads, head_dim,
+                            scale, 0, nullptr, stream);
+}
+
+int ltxattn_check(ltxattn_stream_t stream) {
+  int st;
+  Context* c = current_context(&st);
+  if (!c) return st;
+  return read_and_clear_status(c, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ltxattn_destroy(void) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  Context* c = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_ctx.find(dev);
+    if (it == g_ctx.end()) return LTXATTN_ERR_NOT_INITIALIZED;
+    c = it->second;
+    g_ctx.erase(it);
+  }
+  int st = LTXATTN_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    st = LTXATTN_ERR_CUDA;
+  } else {
+    st = read_and_clear_status(c, nullptr);
+  }
+  for (auto& kv : c->workspaces)
+    if (kv.second.ptr) cudaFree(kv.second.ptr);
+  cudaFree(c->d_status);
+  delete c;
+  return st;
+}
+
+const char* ltxattn_status_string(int status) {
+  switch (status) {
+    case LTXATTN_OK: return "LTXATTN_OK";
+    case LTXATTN_ERR_INVALID_ARG: return "LTXATTN_ERR_INVALID_ARG";
+    case LTXATTN_ERR_UNSUPPORTED: return "LTXATTN_ERR_UNSUPPORTED";
+    case LTXATTN_ERR_MISALIGNED: return "LTXATTN_ERR_MISALIGNED";
+    case LTXATTN_ERR_CUDA: return "LTXATTN_ERR_CUDA";
+    case LTXATTN_ERR_DEVICE_TIMEOUT: return "LTXATTN_ERR_DEVICE_TIMEOUT";
+    case LTXATTN_ERR_NOT_INITIALIZED: return "LTXATTN_ERR_NOT_INITIALIZED";
+    default: return "LTXATTN_UNKNOWN_STATUS";
+  }
+}
+
+int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltxattn_stream_t stream_) {
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull) return LTXATTN_ERR_INVALID_ARG;
+  int st;
+  Context* c = current_context(&st);
+  if (!c) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  st = read_and_clear_status(c, stream);  // start from a clean word
+  if (st == LTXATTN_ERR_CUDA) return st;
+  wait_probe_kernel<<<1, 32, 0, stream>>>(c->d_status, timeout_ns);
+  if (cudaGetLastError() != cudaSuccess) return LTXATTN_ERR_CUDA;
+  return read_and_clear_status(c, stream);
+}
+
+int ltxattn_num_entry_points(void) {
+  return (int)(sizeof(kEntryPoints) / sizeof(kEntryPoints[0]));
+}
+
+const char* ltxattn_entry_point_name(int i) {
+  if (i < 0 || i >= ltxattn_num_entry_points()) return nullptr;
+  return kEntryPoints[i];
+}
+
+}  // extern "C"

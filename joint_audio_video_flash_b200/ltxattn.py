@@ -1,0 +1,132 @@
+"""ctypes binding of libltxattn.so (the C ABI in include/ltxattn.h).
+
+Argument marshalling only: torch tensors are checked for dtype, device, shape and
+contiguity, and their device pointers are passed to the library together with
+the current CUDA stream.  There is no fallback: if the library is missing or a
+call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libltxattn.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "ltxattn.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT, \
+    ERR_NOT_INITIALIZED = range(7)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class LtxAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libltxattn.so (built by ``joint_audio_video_flash_b200.build``); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: run joint_audio_video_flash_b200.build")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            lib.ltxattn_create.argtypes = []
+            lib.ltxattn_forward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, vp]
+            lib.ltxattn_forward_ex.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci,
+                                               ctypes.POINTER(ci), vp]
+            lib.ltxattn_check.argtypes = [vp]
+            lib.ltxattn_destroy.argtypes = []
+            lib.ltxattn_status_string.argtypes = [ci]
+            lib.ltxattn_status_string.restype = ctypes.c_char_p
+            lib.ltxattn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
+            lib.ltxattn_num_entry_points.argtypes = []
+            lib.ltxattn_entry_point_name.argtypes = [ci]
+            lib.ltxattn_entry_point_name.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def header_entry_points() -> list[str]:
+    """Function names declared in include/ltxattn.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"^\s*(?:LTXATTN_API\s+)?(?:int|const char\*)\s+(ltxattn_\w+)\s*\(", text, flags=re.M)
+
+
+def status_string(status: int) -> str:
+    return load().ltxattn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise LtxAttnError(status, where)
+
+
+def create() -> None:
+    _check(load().ltxattn_create(), "ltxattn_create")
+
+
+def destroy() -> None:
+    _check(load().ltxattn_destroy(), "ltxattn_destroy")
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def check(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel recorded a stalled wait."""
+    _check(load().ltxattn_check(ctypes.c_void_p(_stream_handle(stream))), "ltxattn_check")
+
+
+def selftest_wait_timeout(timeout_ns: int = 1_000_000, stream=None) -> int:
+    """Run the bounded-wait self-test; returns the raw status (DEVICE_TIMEOUT expected)."""
+    return int(load().ltxattn_selftest_wait_timeout(ctypes.c_ulonglong(int(timeout_ns)),
+                                                      ctypes.c_void_p(_stream_handle(stream))))
+
+
+def forward(q, k, v, out=None, *, kv_valid_len: int | None = None, scale: float | None = None,
+            num_splits: int = 0, stream=None, return_splits: bool = False):
+    """O = softmax(scale q k^T, keys < kv_valid_len) v for bf16 BSHD CUDA tensors.
+
+    q: [B, Lq, H, D]; k, v: [B, Lkv, H, D]; out (optional): [B, Lq, H, D].
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [batch, len, heads, head_dim] tensor")
+    batch, q_len, heads, head_dim = q.shape
+    kv_len = k.shape[1]
+    if tuple(k.shape) != (batch, kv_len, heads, head_dim) or v.shape != k.shape:
+        raise ValueError("k and v must be [batch, kv_len, heads, head_dim] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    elif (out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous()
+          or out.device != q.device):
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q on q's device")
+    if kv_valid_len is None:
+        kv_valid_len = kv_len
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    used = ctypes.c_int(0)
+    st = load().ltxattn_forward_ex(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()), int(q_len), int(kv_len),
+        int(kv_valid_len), int(batch), int(heads), int(head_dim), ctypes.c_float(scale),
+        int(num_splits), ctypes.byref(used), ctypes.c_void_p(_stream_handle(stream)))
+    _check(st, "ltxattn_forward")
+    return (out, used.value) if return_splits else out

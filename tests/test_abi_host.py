@@ -1,0 +1,93 @@
+"""The C ABI library loads, exports what include/ltxattn.h declares, and rejects bad
+arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+
+import pytest
+
+from joint_audio_video_flash_b200 import build, ltxattn
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ltxattn.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = ltxattn.header_entry_points()
+    assert len(declared) >= 5
+    for name in ("ltxattn_create", "ltxattn_forward", "ltxattn_destroy"):
+        assert name in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    listed = [lib.ltxattn_entry_point_name(i).decode()
+              for i in range(lib.ltxattn_num_entry_points())]
+    assert sorted(listed) == sorted(declared)
+    assert lib.ltxattn_entry_point_name(-1) is None
+    assert lib.ltxattn_entry_point_name(len(listed)) is None
+
+
+def test_status_strings(lib):
+    names = [ltxattn.status_string(i) for i in range(7)]
+    assert names[0] == "LTXATTN_OK"
+    assert names[5] == "LTXATTN_ERR_DEVICE_TIMEOUT"
+    assert len(set(names)) == 7
+    assert ltxattn.status_string(99) == "LTXATTN_UNKNOWN_STATUS"
+
+
+# fake, never dereferenced device addresses: validation fails before any CUDA call
+Q, K, V, O = 1 << 20, 2 << 20, 3 << 20, 4 << 20
+
+
+def fwd(lib, q=Q, k=K, v=V, o=O, q_len=128, kv_len=128, valid=128, batch=2, heads=4, d=64,
+        scale=0.125, splits=None):
+    args = [ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v), ctypes.c_void_p(o),
+            q_len, kv_len, valid, batch, heads, d, ctypes.c_float(scale)]
+    if splits is None:
+        return lib.ltxattn_forward(*args, None)
+    return lib.ltxattn_forward_ex(*args, splits, None, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), ltxattn.ERR_INVALID_ARG),
+    (dict(o=0), ltxattn.ERR_INVALID_ARG),
+    (dict(q_len=0), ltxattn.ERR_INVALID_ARG),
+    (dict(kv_len=0, valid=0), ltxattn.ERR_INVALID_ARG),
+    (dict(valid=0), ltxattn.ERR_INVALID_ARG),
+    (dict(valid=129), ltxattn.ERR_INVALID_ARG),
+    (dict(batch=0), ltxattn.ERR_INVALID_ARG),
+    (dict(heads=-1), ltxattn.ERR_INVALID_ARG),
+    (dict(scale=0.0), ltxattn.ERR_INVALID_ARG),
+    (dict(scale=-1.0), ltxattn.ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ltxattn.ERR_INVALID_ARG),
+    (dict(scale=float("inf")), ltxattn.ERR_INVALID_ARG),
+    (dict(d=96), ltxattn.ERR_UNSUPPORTED),
+    (dict(d=256), ltxattn.ERR_UNSUPPORTED),
+    (dict(q_len=(1 << 24) + 1), ltxattn.ERR_UNSUPPORTED),
+    (dict(heads=1025), ltxattn.ERR_UNSUPPORTED),
+    (dict(batch=1025), ltxattn.ERR_UNSUPPORTED),
+    (dict(q=Q + 8), ltxattn.ERR_MISALIGNED),
+    (dict(k=K + 2), ltxattn.ERR_MISALIGNED),
+    (dict(o=O + 4), ltxattn.ERR_MISALIGNED),
+    (dict(o=Q), ltxattn.ERR_INVALID_ARG),             # out aliases q
+    (dict(o=K + 4096), ltxattn.ERR_INVALID_ARG),      # out overlaps k
+    (dict(splits=-1), ltxattn.ERR_INVALID_ARG),
+])
+def test_host_validation(lib, kw, status):
+    assert fwd(lib, **kw) == status
+
+
+def test_validation_order_invalid_before_unsupported_before_misaligned(lib):
+    assert fwd(lib, valid=0, d=96, q=Q + 2) == ltxattn.ERR_INVALID_ARG
+    assert fwd(lib, d=96, q=Q + 2) == ltxattn.ERR_UNSUPPORTED
+
+
+def test_valid_arguments_reach_cuda(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-only expectation: no CUDA device")
+    # validation passes, then the first CUDA call fails without a device
+    assert fwd(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
+    assert lib.ltxattn_create() == ltxattn.ERR_CUDA
+    assert lib.ltxattn_selftest_wait_timeout(ctypes.c_ulonglong(10), None) == \
+        ltxattn.ERR_INVALID_ARG
