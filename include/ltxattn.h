@@ -144,6 +144,54 @@ LTXATTN_API const char* ltxattn_status_string(int status);
  */
 LTXATTN_API int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltxattn_stream_t stream);
 
+/* Size of the library's built-in scratch array used by ltxattn_forward_split_noalloc. */
+#define LTXATTN_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per GPU */
+
+/*
+ * Key-split attention forward that allocates no memory at all.  (The pages this
+ * library follows have no counterpart to this call; it exists for embedding.)
+ *
+ * Some callers cannot let a library call cudaMalloc: a host framework or plugin
+ * host that owns every byte of device memory and hands out none, a serving loop
+ * that has fixed its memory plan at start-up and must not stall other streams on
+ * the device-wide synchronisation an allocation can cause, or a process running
+ * under a hard device-memory quota.  ltxattn_forward may allocate its key-split
+ * workspace (and ltxattn_create allocates the status word); this call never does.
+ * It needs no ltxattn_create.
+ *
+ * It computes exactly what ltxattn_forward computes, always through the key-range
+ * split path: per-part fp32 partial outputs and base-2 log-sum-exps, merged by
+ * the combine kernel.  Those partials live in one array of
+ * LTXATTN_NOALLOC_SCRATCH_BYTES in the library's own device memory (a static
+ * device array: every GPU that loads the library holds it until the process
+ * exits).  The caller passes inputs and outputs as for ltxattn_forward.
+ *
+ *   num_splits  0 = the library's plan, reduced until the partials fit; >= 1 =
+ *               that many key-range parts (clamped to the number of 128-key tiles).
+ *   Scratch use: 256 + splits * batch * heads * ceil(q_len/128)*128 *
+ *               (head_dim + 1) * 4 bytes must not exceed
+ *               LTXATTN_NOALLOC_SCRATCH_BYTES, else LTXATTN_ERR_UNSUPPORTED is
+ *               returned and nothing is enqueued.
+ *
+ * The first call on each device sets up that device (the scratch array's device
+ * address via cudaGetSymbolAddress, the kernels' shared-memory limits, the
+ * tensor-map encoder); make that first call before any stream capture.
+ * Every call shares the one array and it keeps the last call's contents.  Nothing
+ * in it has to start at zero except the status word in its first 256 bytes, which
+ * each call clears on `stream` before its kernels run; every partial the merge
+ * reads is written earlier in the same call.  Calls whose GPU work overlaps (on
+ * different streams, or from different host threads without ordering) race on the
+ * array and give wrong results: order them.  A kernel wait that runs out is
+ * recorded in that status word only; this call does not report it.
+ * Returns LTXATTN_OK once enqueued, or INVALID_ARG / UNSUPPORTED / MISALIGNED (as
+ * ltxattn_forward, before any CUDA call), UNSUPPORTED when the scratch is too
+ * small, LTXATTN_ERR_CUDA on a failed set-up or launch.
+ */
+LTXATTN_API int ltxattn_forward_split_noalloc(const void* q, const void* k, const void* v,
+                                              void* out, int q_len, int kv_len, int kv_valid_len,
+                                              int batch, int heads, int head_dim, float scale,
+                                              int num_splits, ltxattn_stream_t stream);
+
 /*
  * Number of entry points above, and their names, for loaders that check the
  * exported symbols.

@@ -47,6 +47,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_create",        "ltxattn_forward",          "ltxattn_forward_ex",
     "ltxattn_check",         "ltxattn_destroy",          "ltxattn_status_string",
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
+    "ltxattn_forward_split_noalloc",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -376,3 +377,146 @@ const char* ltxattn_entry_point_name(int i) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free key-split forward (ltxattn_forward_split_noalloc).
+//
+// For callers that may not allocate device memory (a plugin host that owns all
+// of it, a serving loop with a fixed memory plan that must not stall on an
+// allocation's device-wide synchronisation, a hard memory quota), the key-split
+// partials live in this file-scope device array instead of a cudaMalloc'd
+// workspace.  Host code cannot use the array's name as a device address, so the
+// first call on each device looks the address up with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LTXATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+constexpr size_t kNoallocStatusBytes = 256;  // status word at offset 0, partials after it
+
+struct NoallocDevice {
+  bool ready = false;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  int num_sms = 0;
+};
+
+std::mutex g_noalloc_mu;
+NoallocDevice g_noalloc_dev[kNoallocMaxDevices];
+EncodeTiledFn g_noalloc_encode = nullptr;
+
+// Once per device, with that device current: scratch address, SM count, kernel
+// shared-memory limits and the tensor-map encoder.  Allocates nothing.
+int noalloc_setup(int dev, NoallocDevice** out) {
+  if (dev < 0 || dev >= kNoallocMaxDevices) return LTXATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  NoallocDevice& d = g_noalloc_dev[dev];
+  if (!d.ready) {
+    void* sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_noalloc_scratch) != cudaSuccess || sym == nullptr) {
+      cudaGetLastError();
+      return LTXATTN_ERR_CUDA;
+    }
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        set_smem_limits<64>() != cudaSuccess || set_smem_limits<128>() != cudaSuccess) {
+      cudaGetLastError();
+      return LTXATTN_ERR_CUDA;
+    }
+    if (!g_noalloc_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        cudaGetLastError();
+        return LTXATTN_ERR_CUDA;
+      }
+      g_noalloc_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.scratch = static_cast<unsigned char*>(sym);
+    d.ready = true;
+  }
+  *out = &d;
+  return LTXATTN_OK;
+}
+
+size_t noalloc_bytes(int splits, int batch, int heads, int n_q_tiles, int head_dim) {
+  const size_t rows = (size_t)splits * batch * heads * (size_t)n_q_tiles * ltx::kBlockM;
+  return kNoallocStatusBytes + rows * (size_t)(head_dim + 1) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" int ltxattn_forward_split_noalloc(const void* q, const void* k, const void* v,
+                                             void* out, int q_len, int kv_len, int kv_valid_len,
+                                             int batch, int heads, int head_dim, float scale,
+                                             int num_splits, ltxattn_stream_t stream_) {
+  int st = validate(q, k, v, out, q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale);
+  if (st != LTXATTN_OK) return st;
+  if (num_splits < 0) return LTXATTN_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  NoallocDevice* d = nullptr;
+  st = noalloc_setup(dev, &d);
+  if (st != LTXATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+
+  FwdParams p{};
+  p.q_len = q_len;
+  p.kv_len = kv_len;
+  p.kv_valid = kv_valid_len;
+  p.heads = heads;
+  p.batch = batch;
+  p.n_q_tiles = (q_len + ltx::kBlockM - 1) / ltx::kBlockM;
+  p.n_kv_tiles = (kv_valid_len + ltx::kBlockN - 1) / ltx::kBlockN;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kDefaultTimeoutNs;
+
+  int splits;
+  if (num_splits > 0) {
+    splits = std::min(num_splits, p.n_kv_tiles);
+  } else {
+    splits = plan_splits(p.n_q_tiles * heads * batch, p.n_kv_tiles, d->num_sms);
+    while (splits > 1 && noalloc_bytes(splits, batch, heads, p.n_q_tiles, head_dim) >
+                             LTXATTN_NOALLOC_SCRATCH_BYTES)
+      --splits;
+  }
+  p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
+  splits = (p.n_kv_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
+  if (noalloc_bytes(splits, batch, heads, p.n_q_tiles, head_dim) > LTXATTN_NOALLOC_SCRATCH_BYTES)
+    return LTXATTN_ERR_UNSUPPORTED;  // the partials would not fit in the scratch array
+  p.num_splits = splits;
+
+  const size_t rows = (size_t)splits * batch * heads * (size_t)p.n_q_tiles * ltx::kBlockM;
+  p.status = reinterpret_cast<int*>(d->scratch);
+  p.o_part = reinterpret_cast<float*>(d->scratch + kNoallocStatusBytes);
+  p.lse_part = p.o_part + rows * (size_t)head_dim;
+
+  Context c;  // tensor-map encoder only; nothing in it is allocated
+  c.encode = g_noalloc_encode;
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bshd(c, &tq, q, q_len, batch, heads, head_dim) ||
+      !encode_bshd(c, &tk, k, kv_len, batch, heads, head_dim) ||
+      !encode_bshd(c, &tv, v, kv_len, batch, heads, head_dim) ||
+      !encode_bshd(c, &to, out, q_len, batch, heads, head_dim))
+    return LTXATTN_ERR_CUDA;
+
+  // the status word is the one thing that must start at zero
+  if (cudaMemsetAsync(p.status, 0, sizeof(int), stream) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  cudaError_t e;
+  if (head_dim == 64) {
+    e = launch_fwd<64, true>(tq, tk, tv, to, p, stream);
+    if (e == cudaSuccess) e = launch_combine<64>(p, out, stream);
+  } else {
+    e = launch_fwd<128, true>(tq, tk, tv, to, p, stream);
+    if (e == cudaSuccess) e = launch_combine<128>(p, out, stream);
+  }
+  return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}

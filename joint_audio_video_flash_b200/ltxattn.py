@@ -130,3 +130,29 @@ def forward(q, k, v, out=None, *, kv_valid_len: int | None = None, scale: float 
         int(num_splits), ctypes.byref(used), ctypes.c_void_p(_stream_handle(stream)))
     _check(st, "ltxattn_forward")
     return (out, used.value) if return_splits else out
+
+
+def forward_split_noalloc(q, k, v, out, *, kv_valid_len: int | None = None,
+                          scale: float | None = None, num_splits: int = 0, stream=None) -> int:
+    """Key-split forward that allocates no device memory (``ltxattn_forward_split_noalloc``).
+
+    For callers that must not let the library allocate (a plugin host that owns all
+    device memory, a serving loop with a fixed memory plan, a hard memory quota):
+    the fp32 partials go to the library's built-in 16 MiB scratch array.  ``out`` is
+    required (this call allocates nothing, not even the output).  Returns the raw
+    status; calls whose GPU work overlaps race on the shared scratch.
+    """
+    lib = load()
+    fn = lib.ltxattn_forward_split_noalloc
+    vp, ci = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ctypes.c_float, ci, vp]
+    batch, q_len, heads, head_dim = q.shape
+    kv_len = k.shape[1]
+    if kv_valid_len is None:
+        kv_valid_len = kv_len
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    return int(fn(vp(q.data_ptr()), vp(k.data_ptr()), vp(v.data_ptr()), vp(out.data_ptr()),
+                  int(q_len), int(kv_len), int(kv_valid_len), int(batch), int(heads),
+                  int(head_dim), ctypes.c_float(scale), int(num_splits),
+                  vp(_stream_handle(stream))))
