@@ -33,6 +33,24 @@ if ROOT not in sys.path:
 METRIC = "attention TFLOP/s and µs/call per config; % of B200 dense-BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, keyed by
+# the hash of the kernel sources it was taken on; reported as null once the sources change.
+TRAFFIC = {
+    "video_self": {"src": "4a822a9451cff96e", "bytes_per_token": 254.8e6 / 8192,
+                   "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
+}
+KERNEL_SOURCES = ("joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
+                  "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -263,6 +281,12 @@ def run_ltxattn(args):
             if len(splits) < len(calls):
                 splits.append(used)
 
+    if args.once:  # one launch set, no timing: the command the Nsight Compute captures run
+        step()
+        torch.cuda.synchronize()
+        ltxattn.check()
+        print(json.dumps({"workload": args.workload, "once": True, "splits": splits}))
+        return
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize()
@@ -339,8 +363,13 @@ def run_ltxattn(args):
     v_us = statistics.mean(call_us[vi])
     achieved = calls[vi].flops / (v_us * 1e-6) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    tr = TRAFFIC.get(calls[vi].name)
+    traffic = None
+    if tr is not None and tr["src"] == kernel_source_hash():
+        traffic = tr["bytes_per_token"] * calls[vi].batch * calls[vi].q_len
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": "fmha_fwd_sm100<128>",
+                "frac": achieved / peak, "traffic": traffic, "kernel": "fmha_fwd_sm100<128>",
+                "algorithmic_bytes": calls[vi].bytes,
                 "peak_source": f"{peak_src} bf16_tflops_sustained"}
 
     per_call_out = {}
@@ -391,6 +420,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--once", action="store_true",
+                    help="run each call of the workload once and exit (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

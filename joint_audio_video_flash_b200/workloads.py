@@ -81,6 +81,10 @@ def configs() -> dict:
                      "audio self 126->128 masked + v2a + a2v (32x64), back to back on one stream",
                      [Call("video_self", 2, 15360, 15360, 15360, 32, 128, 15360, _seed(4, 0))]
                      + _audio_stream(4, 2, 15360, 128, 126, 1)),
+        "ncu_small": ("profiling case sized for Nsight Compute replays: video self B1 8192 "
+                      "(32x128, 201 MB of inputs) + a2v and v2a at the 768x1280x121 block size",
+                      [Call("video_self", 1, 8192, 8192, 8192, 32, 128, 8192, _seed(6, 0))]
+                      + _audio_stream(6, 2, 15360, 128, 126, 1)[1:]),
         "longclip": ("long clip 1280x704x241 (27280 video tokens), audio 252->256 masked, B2: "
                      "video self (32x128) + audio self + v2a + a2v (32x64)",
                      [Call("video_self", 2, 27280, 27280, 27280, 32, 128, 27280, _seed(5, 0))]
