@@ -39,7 +39,8 @@ TRAFFIC = {
     "video_self": {"src": "4a822a9451cff96e", "bytes_per_token": 254.8e6 / 8192,
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
 }
-KERNEL_SOURCES = ("joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
+KERNEL_SOURCES = ("joint_audio_video_flash_b200/csrc/fmha_fwd_pp.cuh",
+                  "joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
                   "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh")
 
 

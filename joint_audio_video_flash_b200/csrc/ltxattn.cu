@@ -14,6 +14,7 @@
 #include "../../include/ltxattn.h"
 #include "combine.cuh"
 #include "fmha_fwd.cuh"
+#include "fmha_fwd_pp.cuh"
 
 namespace {
 
@@ -137,6 +138,23 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   return cudaGetLastError();
 }
 
+// Two query tiles per CTA (query sides of more than one 128-row tile).
+template <int D, bool kSplit>
+cudaError_t launch_fwd_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
+  dim3 grid((p.n_q_tiles + 1) / 2, p.heads, p.batch * p.num_splits);
+  ltx::fmha_fwd_pp_sm100<D, kSplit><<<grid, ltx::kPPThreads, ltx::PPSmem<D>::kAlloc, stream>>>(
+      tq, tk, tv, to, p);
+  return cudaGetLastError();
+}
+
+template <int D, bool kSplit>
+cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
+  return p.n_q_tiles >= 2 ? launch_fwd_pp<D, kSplit>(tq, tk, tv, to, p, stream)
+                          : launch_fwd<D, kSplit>(tq, tk, tv, to, p, stream);
+}
+
 template <int D>
 cudaError_t launch_combine(const FwdParams& p, void* out, cudaStream_t stream) {
   const long long total = (long long)p.batch * p.q_len * p.heads * (D / 4);
@@ -155,6 +173,17 @@ cudaError_t set_smem_limits() {
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(ltx::fmha_fwd_sm100<D, true>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<D>::kAlloc);
+}
+
+template <int D>
+cudaError_t set_smem_limits_pp() {
+  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_pp_sm100<D, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       ltx::PPSmem<D>::kAlloc);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ltx::fmha_fwd_pp_sm100<D, true>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ltx::PPSmem<D>::kAlloc);
 }
 
 __global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
@@ -213,6 +242,7 @@ int ltxattn_create(void) {
     ok = cudaMalloc(&c->d_status, sizeof(int)) == cudaSuccess &&
          cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
          set_smem_limits<64>() == cudaSuccess && set_smem_limits<128>() == cudaSuccess &&
+         set_smem_limits_pp<64>() == cudaSuccess && set_smem_limits_pp<128>() == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
@@ -288,12 +318,12 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
 
   cudaError_t e;
   if (head_dim == 64) {
-    e = splits > 1 ? launch_fwd<64, true>(tq, tk, tv, to, p, stream)
-                   : launch_fwd<64, false>(tq, tk, tv, to, p, stream);
+    e = splits > 1 ? launch_attention<64, true>(tq, tk, tv, to, p, stream)
+                   : launch_attention<64, false>(tq, tk, tv, to, p, stream);
     if (e == cudaSuccess && splits > 1) e = launch_combine<64>(p, out, stream);
   } else {
-    e = splits > 1 ? launch_fwd<128, true>(tq, tk, tv, to, p, stream)
-                   : launch_fwd<128, false>(tq, tk, tv, to, p, stream);
+    e = splits > 1 ? launch_attention<128, true>(tq, tk, tv, to, p, stream)
+                   : launch_attention<128, false>(tq, tk, tv, to, p, stream);
     if (e == cudaSuccess && splits > 1) e = launch_combine<128>(p, out, stream);
   }
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;

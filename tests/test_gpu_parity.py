@@ -97,6 +97,17 @@ def test_forced_key_splits(oracle, splits):
     assert_parity(got, ref, f"splits={splits}")
 
 
+@pytest.mark.parametrize("d,splits", [(64, 3), (128, 2), (128, 7)])
+def test_forced_key_splits_two_query_tiles(oracle, d, splits):
+    # query side of several tiles (odd count: the last CTA's second tile is empty)
+    q, k, v = synth.make_qkv(2, 300, 2048, 3, d, seed=17, kv_valid=2000)
+    scale = 1.0 / np.sqrt(d)
+    ref = oracle.attention(q, k, v, scale, kv_valid_len=2000)
+    got, used = gpu_run(q, k, v, 2000, scale, num_splits=splits)
+    assert used > 1
+    assert_parity(got, ref, f"d={d} splits={splits}")
+
+
 def test_growing_scores_force_rescales(oracle):
     # keys ordered so that the running max grows tile after tile (exercises the O rescale)
     q, k, v = synth.make_qkv(1, 130, 1024, 2, 128, seed=8)
