@@ -92,10 +92,10 @@ struct FwdSmem {
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
                                                 unsigned long long timeout_ns) {
   const unsigned long long t0 = global_timer_ns();
-  const unsigned long long max_spins = timeout_ns / 4 + 1024;
-  unsigned long long spins = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > timeout_ns || ++spins > max_spins) return false;
+  const unsigned long long max_polls = timeout_ns / 4 + 1024;
+  unsigned long long polls = 0;
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
+    if (global_timer_ns() - t0 > timeout_ns || ++polls > max_polls) return false;
   }
   return true;
 }

@@ -71,23 +71,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of parity `parity` to complete.  Returns false (and raises
-// the abort flag) on timeout or when another role of the CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
-  if (mbar_try_wait(bar, parity)) return true;
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps in
+// hardware until the phase completes or about `hint_ns` pass (used on drain paths).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kWaitSleepNs = 1000000;  // 1 ms per suspended poll
+
+// Waits for the phase of parity `parity` to complete, polling try_wait (measured
+// faster here than suspended polls: the wake-up sits on the softmax/MMA critical
+// path).  Returns false (and raises the abort flag) on timeout, or when another role
+// of the CTA aborted or another CTA recorded an error.
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity,
+                                               const WaitCtl& ctl) {
   const unsigned long long t0 = global_timer_ns();
-  // second bound, independent of the global timer: every polling round costs
-  // well over 4 ns, so this many rounds take longer than timeout_ns
-  const unsigned long long max_spins = ctl.timeout_ns / 4 + 1024;
-  unsigned long long spins = 0;
+  // second bound, independent of the global timer: every poll costs well over 4 ns
+  const unsigned long long max_polls = ctl.timeout_ns / 4 + 1024;
+  unsigned long long polls = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++spins & 63u) == 0) {
+    if ((++polls & 255u) == 0) {
       if (*ctl.abort_flag) return false;
       if (*reinterpret_cast<volatile int*>(ctl.status) != kDevOk) {
         *ctl.abort_flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > ctl.timeout_ns || spins > max_spins) {
+      if (global_timer_ns() - t0 > ctl.timeout_ns || polls > max_polls) {
         atomicCAS(ctl.status, kDevOk, kDevTimeout);
         *ctl.abort_flag = 1;
         return false;
@@ -95,6 +113,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_poll(bar, parity, ctl);
+}
+
+// Same wait with the polling loop out of line, for the single-thread producer and
+// MMA roles whose hot loops then hold no timer registers.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl ctl) {
+  return mbar_wait_poll(bar, parity, ctl);
+}
+
+__device__ __forceinline__ bool mbar_wait_lean(uint32_t bar, uint32_t parity,
+                                               const WaitCtl& ctl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, ctl);
 }
 
 // ----------------------------------------------------------------------------
@@ -279,6 +314,34 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA/ALU pipes instead of the MUFU, for x <= 2^7.  Method: Cody-Waite
+// style range reduction x = n + f with n = round(x) obtained by adding and
+// subtracting the shifter 1.5 * 2^23 (round to nearest in the FADD), f in [-1/2, 1/2];
+// 2^f from a cubic 1 + c1 f + c2 f^2 + c3 f^3 fitted here for minimum maximum
+// relative error on [-1/2, 1/2] with the constant term held at exactly 1
+// (iteratively reweighted least squares; max relative error 1.02e-4, about a
+// twentieth of a bf16 ulp); 2^n applied by adding n << 23 to the bit pattern (the
+// shifted sum's low mantissa bits hold n).  x is clamped at -127, where f = 0 and
+// p = 1 make the bit pattern exactly +0, so -inf (a masked key) gives exactly 0.
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -127.0f);
+  const float shifter = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + shifter;
+  const float n = t - shifter;
+  const float f = x - n;
+  float p = fmaf(0.055008664727211f, f, 0.24221056699752808f);
+  p = fmaf(p, f, 0.6932829022407532f);
+  p = fmaf(p, f, 1.0f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// max(a, b, c) in one instruction (three-input form of max.f32 on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0-15.
