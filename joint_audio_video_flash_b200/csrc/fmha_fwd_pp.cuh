@@ -26,26 +26,6 @@
 
 namespace ltx {
 
-// Softmax tuning knobs (compile time): which pairs of exponentials go to the FMA
-// pipe (pair index & mask == mask; 0 = none), three-input max, split row sums.
-#ifndef LTX_PP_EMU_MASK
-#define LTX_PP_EMU_MASK 0
-#endif
-#ifndef LTX_PP_MAX3
-#define LTX_PP_MAX3 0
-#endif
-#ifndef LTX_PP_SUM4
-#define LTX_PP_SUM4 0
-#endif
-// P published in two 64-key halves (the first half's PV overlaps the second half's
-// exponentials); one arrival per warp instead of one per thread.
-#ifndef LTX_PP_PHALVES
-#define LTX_PP_PHALVES 1
-#endif
-#ifndef LTX_PP_WARP_ARRIVE
-#define LTX_PP_WARP_ARRIVE 0
-#endif
-
 constexpr int kPPThreads = 384;
 constexpr int kPPRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of 8
 constexpr int kPPRegsProducer = 88;  // warps 0-3 after setmaxnreg.dec
@@ -120,8 +100,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(L::bQF + g), 1);
       mbar_init(bar(L::bSF + g), 1);
-      mbar_init(bar(L::bPF + g), LTX_PP_WARP_ARRIVE ? kBlockM / 32 : kBlockM);
-      mbar_init(bar(L::bPF + 2 + g), LTX_PP_WARP_ARRIVE ? kBlockM / 32 : kBlockM);
+      mbar_init(bar(L::bPF + g), kBlockM);      // P keys 0-63 of tile g
+      mbar_init(bar(L::bPF + 2 + g), kBlockM);  // P keys 64-127 of tile g
       mbar_init(bar(L::bOF + g), 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
@@ -218,18 +198,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       };
       // waits for P_g (both halves) and issues its PV; false on a failed wait
       auto pv = [&](int g, int st, bool acc, uint32_t pph) -> bool {
-#if LTX_PP_PHALVES
         if (!mbar_wait_lean(bar(L::bPF + g), pph, ctl)) return false;
         tc_fence_after();
         pv_part(g, st, acc, 0, kBlockN / 32);
         if (!mbar_wait_lean(bar(L::bPF + 2 + g), pph, ctl)) return false;
         tc_fence_after();
         pv_part(g, st, acc, kBlockN / 32, kBlockN / 16);
-#else
-        if (!mbar_wait_lean(bar(L::bPF + g), pph, ctl)) return false;
-        tc_fence_after();
-        pv_part(g, st, acc, 0, kBlockN / 16);
-#endif
         return true;
       };
       bool ok = mbar_wait_lean(bar(L::bKF + 0), 0, ctl) && mbar_wait_lean(bar(L::bQF + 0), 0, ctl);
@@ -304,22 +278,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int c = 0; c < kBlockN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-#if LTX_PP_MAX3
-      // row max: four independent chains of three-input max
-      float a0 = s[0], a1 = s[32], a2 = s[64], a3 = s[96];
-#pragma unroll
-      for (int t = 1; t < 31; t += 2) {
-        a0 = fmax3(a0, s[t], s[t + 1]);
-        a1 = fmax3(a1, s[32 + t], s[33 + t]);
-        a2 = fmax3(a2, s[64 + t], s[65 + t]);
-        a3 = fmax3(a3, s[96 + t], s[97 + t]);
-      }
-      float mx = fmax3(fmax3(a0, s[31], s[63]), fmax3(a1, s[95], s[127]), fmaxf(a2, a3));
-#else
       float mx = s[0];
 #pragma unroll
       for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
-#endif
       mx *= sl2;
       if (j == 0) {
         m_run = mx;
@@ -342,42 +303,24 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         m_run = mx;
       }
       const float neg_m = -m_run;
-      // exponentials on the MUFU, optionally some pairs on the FMA pipe (exp2_poly3);
-      // row sum in four independent chains
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // exponentials on the MUFU; P is published to the MMA warp in two 64-key halves so
+      // the PV of the first half overlaps the exponentials of the second
+      float sum = 0.0f;
 #pragma unroll
       for (int c = 0; c < kBlockN / 64; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          const float x0 = fmaf(s[c * 64 + 2 * x], sl2, neg_m);
-          const float x1 = fmaf(s[c * 64 + 2 * x + 1], sl2, neg_m);
-          float p0, p1;
-          if (LTX_PP_EMU_MASK != 0 && (x & LTX_PP_EMU_MASK) == LTX_PP_EMU_MASK) {
-            p0 = exp2_poly3(x0);
-            p1 = exp2_poly3(x1);
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          sum4[LTX_PP_SUM4 ? (x & 3) : 0] += p0 + p1;
+          const float p0 = ex2(fmaf(s[c * 64 + 2 * x], sl2, neg_m));
+          const float p1 = ex2(fmaf(s[c * 64 + 2 * x + 1], sl2, neg_m));
+          sum += p0 + p1;
           pk[x] = pack_bf16x2(p0, p1);
         }
         tmem_st32(trow + colS + c * 32, pk);
-        if (LTX_PP_PHALVES || c == kBlockN / 64 - 1) {
-          // publish this half (or the whole row) of P to the MMA warp
-          tmem_st_wait();
-          tc_fence_before();
-          const int pb = LTX_PP_PHALVES ? c * 2 + g : g;
-#if LTX_PP_WARP_ARRIVE
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::bPF + pb));
-#else
-          mbar_arrive(bar(L::bPF + pb));
-#endif
-        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::bPF + c * 2 + g));
       }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run += sum;
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOF + g), 0, ctl));

@@ -316,34 +316,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes instead of the MUFU, for x <= 2^7.  Method: Cody-Waite
-// style range reduction x = n + f with n = round(x) obtained by adding and
-// subtracting the shifter 1.5 * 2^23 (round to nearest in the FADD), f in [-1/2, 1/2];
-// 2^f from a cubic 1 + c1 f + c2 f^2 + c3 f^3 fitted here for minimum maximum
-// relative error on [-1/2, 1/2] with the constant term held at exactly 1
-// (iteratively reweighted least squares; max relative error 1.02e-4, about a
-// twentieth of a bf16 ulp); 2^n applied by adding n << 23 to the bit pattern (the
-// shifted sum's low mantissa bits hold n).  x is clamped at -127, where f = 0 and
-// p = 1 make the bit pattern exactly +0, so -inf (a masked key) gives exactly 0.
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -127.0f);
-  const float shifter = 12582912.0f;  // 1.5 * 2^23
-  const float t = x + shifter;
-  const float n = t - shifter;
-  const float f = x - n;
-  float p = fmaf(0.055008664727211f, f, 0.24221056699752808f);
-  p = fmaf(p, f, 0.6932829022407532f);
-  p = fmaf(p, f, 1.0f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
-// max(a, b, c) in one instruction (three-input form of max.f32 on sm_100).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits 0-15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
