@@ -15,6 +15,7 @@
 #include "combine.cuh"
 #include "fmha_fwd.cuh"
 #include "fmha_fwd_pp.cuh"
+#include "fmha_fwd_skv.cuh"
 
 namespace {
 
@@ -155,6 +156,22 @@ cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const
                           : launch_fwd<D, kSplit>(tq, tk, tv, to, p, stream);
 }
 
+// Short key side (every valid key in at most two 128-key tiles, head_dim 64):
+// persistent CTAs, one per SM, each walking a contiguous run of query tiles.
+bool use_short_kv(const FwdParams& p, int head_dim) {
+  return head_dim == ltx::kSkvD && p.num_splits == 1 && p.n_kv_tiles <= ltx::kSkvMaxKvTiles;
+}
+
+cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdParams& p, int num_sms,
+                       cudaStream_t stream) {
+  const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
+  const int grid = (int)std::min<long long>(total, num_sms);
+  ltx::fmha_fwd_skv_sm100<<<grid, ltx::kSkvThreads, ltx::SkvSmem::kAlloc, stream>>>(tq, tk, tv,
+                                                                                     to, p);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_combine(const FwdParams& p, void* out, cudaStream_t stream) {
   const long long total = (long long)p.batch * p.q_len * p.heads * (D / 4);
@@ -184,6 +201,11 @@ cudaError_t set_smem_limits_pp() {
   return cudaFuncSetAttribute(ltx::fmha_fwd_pp_sm100<D, true>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               ltx::PPSmem<D>::kAlloc);
+}
+
+cudaError_t set_smem_limits_skv() {
+  return cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<false>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, ltx::SkvSmem::kAlloc);
 }
 
 __global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
@@ -243,6 +265,7 @@ int ltxattn_create(void) {
          cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
          set_smem_limits<64>() == cudaSuccess && set_smem_limits<128>() == cudaSuccess &&
          set_smem_limits_pp<64>() == cudaSuccess && set_smem_limits_pp<128>() == cudaSuccess &&
+         set_smem_limits_skv() == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
@@ -317,7 +340,9 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   }
 
   cudaError_t e;
-  if (head_dim == 64) {
+  if (use_short_kv(p, head_dim)) {
+    e = launch_skv(tq, tk, tv, to, p, c->num_sms, stream);
+  } else if (head_dim == 64) {
     e = splits > 1 ? launch_attention<64, true>(tq, tk, tv, to, p, stream)
                    : launch_attention<64, false>(tq, tk, tv, to, p, stream);
     if (e == cudaSuccess && splits > 1) e = launch_combine<64>(p, out, stream);

@@ -87,6 +87,26 @@ def test_ragged_shapes_full(oracle, shape):
     assert_parity(got, oracle.attention(q, k, v, scale, kv_valid_len=valid), str(shape))
 
 
+SHORT_KV_WALKS = [
+    # more (batch, head, query tile) units than SMs: persistent CTAs cross head
+    # boundaries, reloading K/V; one query tile per head makes every tile a new head
+    (4, 64, 128, 128, 126),
+    (3, 50, 200, 256, 252),
+    # eight query tiles per head, two key tiles with the second holding one valid key
+    (2, 16, 1000, 256, 129),
+    (1, 40, 2000, 300, 256),
+]
+
+
+@pytest.mark.parametrize("shape", SHORT_KV_WALKS, ids=lambda s: "b{}h{}_q{}_kv{}v{}".format(*s))
+def test_short_kv_persistent_walks(oracle, shape):
+    b, h, lq, lkv, valid = shape
+    q, k, v = synth.make_qkv(b, lq, lkv, h, 64, seed=31 + lq + h, kv_valid=valid)
+    got, used = gpu_run(q, k, v, valid, 0.125)
+    assert used == 1
+    assert_parity(got, oracle.attention(q, k, v, 0.125, kv_valid_len=valid), str(shape))
+
+
 @pytest.mark.parametrize("splits", [1, 2, 3, 5, 16, 40])
 def test_forced_key_splits(oracle, splits):
     # v2a-like: few query rows, many keys; 2000 valid keys = 16 tiles (ragged last one)
