@@ -87,6 +87,86 @@ struct FwdSmem {
   static constexpr uint32_t kTmemCols = 512;
 };
 
+// ---------------------------------------------------------------------------
+// softmax row helpers (one query row per thread, scores in registers)
+// ---------------------------------------------------------------------------
+// Sets scores of keys >= `valid` to -inf in NC 32-column chunks (key 0 = s[0]).  Only
+// the chunk holding the boundary pays per-element selects; the branches are uniform.
+template <int NC>
+__device__ __forceinline__ void mask_keys(float* s, int valid) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    if (valid <= c * 32) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x) s[c * 32 + x] = -INFINITY;
+    } else if (valid < c * 32 + 32) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        if (c * 32 + x >= valid) s[c * 32 + x] = -INFINITY;
+    }
+  }
+}
+
+// Maximum of N scores: four chains of three-input max.
+template <int N>
+__device__ __forceinline__ float row_max(const float* s) {
+  static_assert(N % 8 == 0 && N >= 16, "row length");
+  float m[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+  for (int c = 4; c + 8 <= N - 4; c += 8)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) m[x] = fmax3(m[x], s[c + x], s[c + 4 + x]);
+  // s[0 .. 4) seeded the chains and the loop consumed s[4 .. N-4); the last four remain
+#pragma unroll
+  for (int x = 0; x < 4; ++x) m[x] = fmaxf(m[x], s[N - 4 + x]);
+  return fmax3(fmaxf(m[0], m[1]), m[2], m[3]);
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe instead of the MUFU (which the
+// exponentials of attention keep saturated on sm_100).  Range reduction x = n + f with
+// n = round(x), obtained by adding and subtracting the shifter 1.5 * 2^23 (the FADD
+// rounds to nearest), f in [-1/2, 1/2]; 2^f from the cubic 1 + c1 f + c2 f^2 + c3 f^3
+// whose coefficients are the minimax fit of the relative error on [-1/2, 1/2] with the
+// constant term held at 1 (linear programming on a dense grid; max relative error
+// 1.01e-4 in fp32 Horner form, a twentieth of a bf16 ulp); 2^n applied by adding n << 23
+// to the bit pattern (the shifted sum's low mantissa bits hold n).  x is clamped at
+// -127, where f = 0 and p = 1 give the bit pattern of +0, so a masked key (-inf)
+// yields exactly 0.  Valid for x <= 127.
+__device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC1 = 0.6932829f, kC2 = 0.24221097f, kC3 = 0.05500906f;
+  x = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);  // x - n, exact
+  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// 32 scores -> p = 2^(s*scale_log2 - m) as 16 packed bf16 pairs; the fp32 p are added
+// to the two packed row-sum accumulators.  Argument and sums use packed fp32 pairs.
+// kFmaEvery > 0 moves every kFmaEvery-th pair's exponentials from the MUFU to the FMA
+// pipe (exp2_fma_pair).
+template <int kFmaEvery = 0>
+__device__ __forceinline__ void exp2_pack16(const float* s, float2 sc2, float2 nm2, float2& la,
+                                            float2& lb, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int x = 0; x < 16; ++x) {
+    const float2 a = __ffma2_rn(make_float2(s[2 * x], s[2 * x + 1]), sc2, nm2);
+    const float2 e = (kFmaEvery > 0 && x % (kFmaEvery > 0 ? kFmaEvery : 1) == kFmaEvery - 1)
+                         ? exp2_fma_pair(a)
+                         : make_float2(ex2(a.x), ex2(a.y));
+    if (x & 1)
+      lb = __fadd2_rn(lb, e);
+    else
+      la = __fadd2_rn(la, e);
+    pk[x] = pack_bf16x2(e.x, e.y);
+  }
+}
+
 // Bounded wait that ignores the abort flag (used to drain copies / MMAs on the
 // abort path before the CTA releases shared and tensor memory).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
@@ -203,19 +283,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
       bool ok = mbar_wait(bar(L::bQ), 0, ctl);
       bool issued = false;
+      // shared-memory descriptors built once; each MMA moves them by an offset
+      const SmemDesc dq = SmemDesc::sw128(sbase + L::kQ, 16, 1024);
+      const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
+      const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, L::kBoxBytes, 1024);
       auto pv = [&](int t) -> bool {
         const int sb = t & 1;
         if (!mbar_wait(bar(L::bPF + sb), (uint32_t)(t >> 1) & 1u, ctl)) return false;
         const int st = t % L::kStages;
         if (!mbar_wait(bar(L::bVF + st), (uint32_t)(t / L::kStages) & 1u, ctl)) return false;
         tc_fence_after();
-        const uint32_t v_base = sbase + L::kV + st * L::kTileBytes;
+        const uint32_t v_off = (uint32_t)st * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
           // B = V tile, N = D (MN-major: d contiguous), K = 16 keys starting at kk*16
-          const uint64_t bdesc = smem_desc_sw128(v_base + kk * 16 * 128, L::kBoxBytes, 1024);
-          umma_ts(tmem + L::kColO, tmem + sb * 128 + kk * 8, bdesc, idesc_pv,
-                  (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + L::kColO, tmem + sb * 128 + kk * 8, dv.at(v_off + kk * 16 * 128),
+                  idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(L::bVE + st));
         umma_commit(bar(L::bOD));
@@ -227,13 +310,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int sb = j & 1;
-        const uint32_t k_base = sbase + L::kK + st * L::kTileBytes;
+        const uint32_t k_off = (uint32_t)st * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(sbase + L::kQ + off, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_base + off, 16, 1024);
-          umma_ss(tmem + sb * 128, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + sb * 128, dq.at(off), dk.at(k_off + off), idesc_qk, kk > 0 ? 1u : 0u);
         }
         issued = true;
         umma_commit(bar(L::bSF + sb));

@@ -32,6 +32,8 @@ constexpr int kPPRegsProducer = 88;  // warps 0-3 after setmaxnreg.dec
 constexpr int kPPRegsSoftmax = 208;  // warps 4-11 after setmaxnreg.inc
 static_assert(128 * kPPRegsProducer + 256 * kPPRegsSoftmax <= kPPThreads * kPPRegsLaunch,
               "register split exceeds the launch allocation");
+// every kPPExp2FmaEvery-th pair of exponentials runs on the FMA pipe (0 = none)
+constexpr int kPPExp2FmaEvery = 0;
 
 template <int D>
 struct PPSmem {
@@ -171,81 +173,89 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mbar_wait_drain(bar(L::bQF + 0), 0, p.timeout_ns);
         mbar_wait_drain(bar(L::bQF + 1), 0, p.timeout_ns);
       }
-    } else if (warp == 1 && lane == 0 && !*abort_flag) {
+    } else if (warp == 1 && !*abort_flag) {
       // ---------------------------------------------------------- MMA issuer
+      // The whole warp runs this loop (control values stay warp-uniform); one elected
+      // lane issues each MMA and commit, and the lanes agree on every wait.
+      auto wt = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait_lean(bar_addr, parity, ctl));
+      };
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
       bool issued = false;
+      // shared-memory descriptors built once; each MMA moves them by an offset
+      const SmemDesc dq = SmemDesc::sw128(sbase + L::kQ, 16, 1024);
+      const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
+      const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, L::kBoxBytes, 1024);
       auto qk = [&](int g, int st) {
-        const uint32_t q_base = sbase + L::kQ + g * L::kTileBytes;
-        const uint32_t k_base = sbase + L::kK + st * L::kTileBytes;
+        const uint32_t q_off = (uint32_t)g * L::kTileBytes;
+        const uint32_t k_off = (uint32_t)st * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          umma_ss(tmem + L::kColS + 128 * g, smem_desc_sw128(q_base + off, 16, 1024),
-                  smem_desc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss_elect(tmem + L::kColS + 128 * g, dq.at(q_off + off), dk.at(k_off + off), idesc_qk,
+                  kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar(L::bSF + g));
+        umma_commit_elect(bar(L::bSF + g));
       };
       // O_g (+)= P_g[:, keys kk0*16 .. kk1*16) V[keys, :]
       auto pv_part = [&](int g, int st, bool acc, int kk0, int kk1) {
-        const uint32_t v_base = sbase + L::kV + st * L::kTileBytes;
+        const uint32_t v_off = (uint32_t)st * L::kTileBytes;
 #pragma unroll
         for (int kk = kk0; kk < kk1; ++kk)
-          umma_ts(tmem + L::kColO + D * g, tmem + L::kColS + 128 * g + kk * 8,
-                  smem_desc_sw128(v_base + kk * 16 * 128, L::kBoxBytes, 1024), idesc_pv,
-                  (acc || kk > 0) ? 1u : 0u);
+          umma_ts_elect(tmem + L::kColO + D * g, tmem + L::kColS + 128 * g + kk * 8,
+                  dv.at(v_off + kk * 16 * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
       // waits for P_g (both halves) and issues its PV; false on a failed wait
       auto pv = [&](int g, int st, bool acc, uint32_t pph) -> bool {
-        if (!mbar_wait_lean(bar(L::bPF + g), pph, ctl)) return false;
+        if (!wt(bar(L::bPF + g), pph)) return false;
         tc_fence_after();
         pv_part(g, st, acc, 0, kBlockN / 32);
-        if (!mbar_wait_lean(bar(L::bPF + 2 + g), pph, ctl)) return false;
+        if (!wt(bar(L::bPF + 2 + g), pph)) return false;
         tc_fence_after();
         pv_part(g, st, acc, kBlockN / 32, kBlockN / 16);
         return true;
       };
-      bool ok = mbar_wait_lean(bar(L::bKF + 0), 0, ctl) && mbar_wait_lean(bar(L::bQF + 0), 0, ctl);
+      bool ok = wt(bar(L::bKF + 0), 0) && wt(bar(L::bQF + 0), 0);
       if (ok) {
         tc_fence_after();
         qk(0, 0);
         issued = true;
-        ok = mbar_wait_lean(bar(L::bQF + 1), 0, ctl);
+        ok = wt(bar(L::bQF + 1), 0);
       }
       if (ok) {
         tc_fence_after();
         qk(1, 0);
-        umma_commit(bar(L::bKE + 0));
+        umma_commit_elect(bar(L::bKE + 0));
       }
       for (int j = 1; j < n && ok; ++j) {
         const int sk = j % L::kStages;
         const int sv = (j - 1) % L::kStages;
         const uint32_t pph = (uint32_t)(j - 1) & 1u;
-        ok = mbar_wait_lean(bar(L::bKF + sk), (uint32_t)(j / L::kStages) & 1u, ctl) &&
-             mbar_wait_lean(bar(L::bVF + sv), (uint32_t)((j - 1) / L::kStages) & 1u, ctl) &&
+        ok = wt(bar(L::bKF + sk), (uint32_t)(j / L::kStages) & 1u) &&
+             wt(bar(L::bVF + sv), (uint32_t)((j - 1) / L::kStages) & 1u) &&
              pv(0, sv, j > 1, pph);
         if (!ok) break;
         qk(0, sk);
         ok = pv(1, sv, j > 1, pph);
         if (!ok) break;
-        umma_commit(bar(L::bVE + sv));
+        umma_commit_elect(bar(L::bVE + sv));
         qk(1, sk);
-        umma_commit(bar(L::bKE + sk));
+        umma_commit_elect(bar(L::bKE + sk));
       }
       if (ok) {
         const int sv = (n - 1) % L::kStages;
         const uint32_t pph = (uint32_t)(n - 1) & 1u;
-        ok = mbar_wait_lean(bar(L::bVF + sv), (uint32_t)((n - 1) / L::kStages) & 1u, ctl) &&
+        ok = wt(bar(L::bVF + sv), (uint32_t)((n - 1) / L::kStages) & 1u) &&
              pv(0, sv, n > 1, pph);
         if (ok) {
-          umma_commit(bar(L::bOF + 0));
+          umma_commit_elect(bar(L::bOF + 0));
           ok = pv(1, sv, n > 1, pph);
         }
-        if (ok) umma_commit(bar(L::bOF + 1));
+        if (ok) umma_commit_elect(bar(L::bOF + 1));
       }
       if (!ok && issued) {
-        umma_commit(bar(L::bDrain));
+        umma_commit_elect(bar(L::bDrain));
         mbar_wait_drain(bar(L::bDrain), 0, p.timeout_ns);
       }
     }
@@ -272,16 +282,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         tmem_ld32(trow + colS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
       tmem_ld_wait();
       const int kv0 = (kv_begin + j) * kBlockN;
-      if (kv0 + kBlockN > p.kv_valid) {
+      if (kv0 + kBlockN > p.kv_valid) {  // last key tile only
         const int lim = p.kv_valid - kv0;
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
-      mx *= sl2;
+      float mx = row_max<kBlockN>(s) * sl2;
       if (j == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, mx > m_run + kRescaleThreshold)) {
@@ -302,26 +309,24 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         l_run *= f;
         m_run = mx;
       }
-      const float neg_m = -m_run;
-      // exponentials on the MUFU; P is published to the MMA warp in two 64-key halves so
-      // the PV of the first half overlaps the exponentials of the second
-      float sum = 0.0f;
+      const float2 nm2 = make_float2(-m_run, -m_run);
+      const float2 sc2 = make_float2(sl2, sl2);
+      // exponentials on the MUFU (argument and row sum in packed fp32 pairs); P is
+      // published to the MMA warp in two 64-key halves so the PV of the first half
+      // overlaps the exponentials of the second
+      float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int c = 0; c < kBlockN / 64; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float p0 = ex2(fmaf(s[c * 64 + 2 * x], sl2, neg_m));
-          const float p1 = ex2(fmaf(s[c * 64 + 2 * x + 1], sl2, neg_m));
-          sum += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(trow + colS + c * 32, pk);
+        uint32_t pk0[16], pk1[16];
+        exp2_pack16<kPPExp2FmaEvery>(&s[c * 64], sc2, nm2, la, lb, pk0);
+        exp2_pack16<kPPExp2FmaEvery>(&s[c * 64 + 32], sc2, nm2, la, lb, pk1);
+        tmem_st16(trow + colS + c * 32, pk0);
+        tmem_st16(trow + colS + c * 32 + 16, pk1);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::bPF + c * 2 + g));
       }
-      l_run += sum;
+      l_run += (la.x + la.y) + (lb.x + lb.y);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOF + g), 0, ctl));
     ok = named_bar_and(1 + g, kBlockM, ok && !*abort_flag);

@@ -3,47 +3,68 @@
 // audio self-attention of an LTX-2 block ("LTX-2: replicate audio stream across
 // Ulysses ranks by default", Description).  Same operation, layout and key mask as
 // fmha_fwd.cuh.  With every key in one S tile the softmax max is exact, so there is
-// no online rescale.  The work is bound by HBM (reading Q, writing O), so the design
-// keeps loads and stores in flight instead of optimising the (small) MMAs:
+// no online rescale.  The work is bound by HBM (reading Q, writing O) and by the
+// exponentials, so the design keeps both busy at once:
 //
 //   - persistent: one CTA per SM walks a contiguous run of query tiles (flattened
 //     over batch, head, tile); K and V of the current (batch, head) stay resident in
 //     shared memory and are reloaded only when the run crosses into the next head;
-//   - warp 0 streams Q tiles through a 4-stage TMA ring;
-//   - warp 1 issues S = Q K^T (one M=128, N=128*n_kv MMA chain) for tile i+1 before
-//     O = P V of tile i, so QK overlaps the softmax;
-//   - two softmax warpgroups take alternate tiles, each with its own TMEM buffer
-//     (S / P / O) and its own output staging buffer for the TMA store.
-// TMEM (512 columns): buffer b at 256*b: S at [0, 128*n_kv), P packed over its first
-// 64*n_kv columns, O at [128, 192) (for n_kv = 2 O reuses S columns the softmax has
-// already read).
+//   - warp 0 streams Q tiles through a deep TMA ring (8 stages for one key tile);
+//   - warp 1 issues S = Q K^T two tiles ahead of O = P V, so a softmax warpgroup
+//     finds its next scores computed when it finishes a tile;
+//   - warps 4-11: two softmax warpgroups take alternate tiles (S -> P and the row
+//     sum l); they never wait for the PV product;
+//   - warps 12-15: the epilogue warpgroup takes every tile in order: waits for O,
+//     divides by l, rounds to bf16, stages the tile (two staging buffers) and
+//     issues its TMA store.
+// TMEM (512 columns) holds NB = 4 / NKV buffers of 128*NKV columns; tile i uses buffer
+// i % NB.  In a buffer: S over all 128*NKV columns, P packed as bf16 pairs over the
+// first 64*NKV columns (written after the scores it replaces were read), O (64 fp32
+// columns) right after P, over scores already read.
+// Registers (setmaxnreg): producer/MMA warpgroup 56, epilogue 104, softmax 176.
 #pragma once
 
 #include "fmha_fwd.cuh"
 
 namespace ltx {
 
-constexpr int kSkvThreads = 384;
+constexpr int kSkvThreads = 512;
 constexpr int kSkvD = 64;
 constexpr int kSkvMaxKvTiles = 2;
+constexpr int kSkvRegsLaunch = 128;  // 65536 / 512
+constexpr int kSkvRegsIssue = 56;    // warps 0-3
+constexpr int kSkvRegsEpi = 104;     // warps 12-15
+constexpr int kSkvRegsSoftmax = 176; // warps 4-11
+static_assert(128 * kSkvRegsIssue + 128 * kSkvRegsEpi + 256 * kSkvRegsSoftmax <=
+                  kSkvThreads * kSkvRegsLaunch,
+              "register split exceeds the launch allocation");
 
+template <int NKV>
 struct SkvSmem {
+  static_assert(NKV == 1 || NKV == 2, "one or two 128-key tiles");
   static constexpr int kBoxBytes = kBlockM * 128;  // 128 rows x 64 bf16
-  static constexpr int kQStages = 4;
-  static constexpr int kK = 0;                                  // up to 2 key tiles
-  static constexpr int kV = kK + kSkvMaxKvTiles * kBoxBytes;
-  static constexpr int kQ = kV + kSkvMaxKvTiles * kBoxBytes;     // Q ring
-  static constexpr int kStage = kQ + kQStages * kBoxBytes;       // 2 output staging
-  static constexpr int kBar = kStage + 2 * kBoxBytes;
+  static constexpr int kQStages = NKV == 1 ? 8 : 6;
+  static constexpr int kNB = 4 / NKV;                   // TMEM buffers
+  // QK runs this many tiles ahead of PV; QK(i + kLookahead) reuses the buffer of tile
+  // i + kLookahead - kNB, whose epilogue needs PV(i + kLookahead - kNB) issued earlier
+  static constexpr int kLookahead = kNB - 1 < 2 ? kNB - 1 : 2;
+  static constexpr uint32_t kBufCols = 128u * NKV;      // columns per buffer
+  static constexpr uint32_t kColO = 64u * NKV;          // O within a buffer (after P)
+  static constexpr int kK = 0;                          // NKV key tiles
+  static constexpr int kV = kK + NKV * kBoxBytes;
+  static constexpr int kQ = kV + NKV * kBoxBytes;       // Q ring
+  static constexpr int kStage = kQ + kQStages * kBoxBytes;  // 2 output staging buffers
+  static constexpr int kRowSum = kStage + 2 * kBoxBytes;    // l per buffer and row (fp32)
+  static constexpr int kBar = kRowSum + kNB * kBlockM * 4;
   static constexpr int bKVF = 0;
   static constexpr int bKVE = 1;
   static constexpr int bQF = 2;                 // kQStages
   static constexpr int bQE = bQF + kQStages;    // kQStages
-  static constexpr int bSF = bQE + kQStages;    // 2
-  static constexpr int bPF = bSF + 2;           // 2
-  static constexpr int bOF = bPF + 2;           // 2
-  static constexpr int bTF = bOF + 2;           // 2: TMEM buffer free
-  static constexpr int bDrain = bTF + 2;
+  static constexpr int bSF = bQE + kQStages;    // kNB
+  static constexpr int bPF = bSF + kNB;         // kNB
+  static constexpr int bOF = bPF + kNB;         // kNB
+  static constexpr int bTF = bOF + kNB;         // kNB: TMEM buffer free
+  static constexpr int bDrain = bTF + kNB;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
@@ -52,17 +73,51 @@ struct SkvSmem {
                                     ? ((kUsed + 1024 + 1023) / 1024) * 1024
                                     : kMinSmemFor1Cta;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColO = 128;  // within a 256-column buffer
+  static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
+  static_assert(kLookahead >= 1 && kLookahead <= kNB - 1 && kLookahead < kQStages,
+                "pipeline depth");
 };
 
-template <bool kUnused = false>
+// (batch, head, query tile) of consecutive flattened tile indices, advanced without
+// division.
+struct SkvCursor {
+  int b, h, qt;
+  __device__ __forceinline__ void init(long long t, const FwdParams& p) {
+    const long long bh = t / p.n_q_tiles;
+    qt = (int)(t - bh * p.n_q_tiles);
+    b = (int)(bh / p.heads);
+    h = (int)(bh - (long long)b * p.heads);
+  }
+  // true when the next tile starts another (batch, head)
+  __device__ __forceinline__ bool advance(const FwdParams& p) {
+    if (++qt < p.n_q_tiles) return false;
+    qt = 0;
+    if (++h == p.heads) {
+      h = 0;
+      ++b;
+    }
+    return true;
+  }
+};
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
+}
+
+template <int NKV>
 __global__ void __launch_bounds__(kSkvThreads, 1)
     fmha_fwd_skv_sm100(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
-  using L = SkvSmem;
+  using L = SkvSmem<NKV>;
   constexpr int D = kSkvD;
+  constexpr int NB = L::kNB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -70,17 +125,15 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  float* row_sum = reinterpret_cast<float*>(smem + L::kRowSum);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_kv = p.n_kv_tiles;  // 1 or 2
   // contiguous run of flattened (batch, head, query tile) indices for this CTA
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
   const long long t_begin = total * blockIdx.x / gridDim.x;
   const long long t_end = total * (blockIdx.x + 1) / gridDim.x;
   const int cnt = (int)(t_end - t_begin);
-  auto tile_bh = [&](int i) -> int { return (int)((t_begin + i) / p.n_q_tiles); };
-  auto tile_qt = [&](int i) -> int { return (int)((t_begin + i) % p.n_q_tiles); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::bKVF), 1);
@@ -89,11 +142,11 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       mbar_init(bar(L::bQF + s), 1);
       mbar_init(bar(L::bQE + s), 1);
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(bar(L::bSF + g), 1);
-      mbar_init(bar(L::bPF + g), kBlockM);
-      mbar_init(bar(L::bOF + g), 1);
-      mbar_init(bar(L::bTF + g), kBlockM);
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(bar(L::bSF + b), 1);
+      mbar_init(bar(L::bPF + b), kBlockM);
+      mbar_init(bar(L::bOF + b), 1);
+      mbar_init(bar(L::bTF + b), kBlockM);
     }
     mbar_init(bar(L::bDrain), 1);
     *abort_flag = (*reinterpret_cast<volatile int*>(p.status) != kDevOk) ? 1 : 0;
@@ -109,39 +162,44 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
 
+  // The register split (setmaxnreg) sits inside each role's branch, so that ptxas
+  // compiles every role under the limit it runs with.
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    setmaxnreg_dec<kSkvRegsIssue>();
     if (lane == 0 && !*abort_flag && cnt > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int cur_bh = -1, kv_loads = 0;
+      SkvCursor cur;
+      cur.init(t_begin, p);
+      int kv_loads = 0;
+      bool new_head = true;
       int last_q[L::kQStages];
       for (int s = 0; s < L::kQStages; ++s) last_q[s] = -1;
       bool ok = true;
       for (int i = 0; i < cnt && ok; ++i) {
-        const int bh = tile_bh(i);
-        const int b = bh / p.heads, h = bh % p.heads;
-        if (bh != cur_bh) {
+        if (new_head) {
           if (kv_loads > 0) ok = mbar_wait_lean(bar(L::bKVE), (uint32_t)(kv_loads - 1) & 1u, ctl);
           if (!ok) break;
-          mbar_arrive_expect_tx(bar(L::bKVF), 2 * n_kv * L::kBoxBytes);
-          for (int t = 0; t < n_kv; ++t) {
-            tma_load_4d(sbase + L::kK + t * L::kBoxBytes, &tm_k, bar(L::bKVF), 0, h,
-                        t * kBlockN, b);
-            tma_load_4d(sbase + L::kV + t * L::kBoxBytes, &tm_v, bar(L::bKVF), 0, h,
-                        t * kBlockN, b);
+          mbar_arrive_expect_tx(bar(L::bKVF), 2 * NKV * L::kBoxBytes);
+#pragma unroll
+          for (int t = 0; t < NKV; ++t) {
+            tma_load_4d(sbase + L::kK + t * L::kBoxBytes, &tm_k, bar(L::bKVF), 0, cur.h,
+                        t * kBlockN, cur.b);
+            tma_load_4d(sbase + L::kV + t * L::kBoxBytes, &tm_v, bar(L::bKVF), 0, cur.h,
+                        t * kBlockN, cur.b);
           }
-          cur_bh = bh;
           ++kv_loads;
         }
         const int qs = i % L::kQStages;
         ok = mbar_wait_lean(bar(L::bQE + qs), ((uint32_t)(i / L::kQStages) & 1u) ^ 1u, ctl);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(L::bQF + qs), L::kBoxBytes);
-        tma_load_4d(sbase + L::kQ + qs * L::kBoxBytes, &tm_q, bar(L::bQF + qs), 0, h,
-                    tile_qt(i) * kBlockM, b);
+        tma_load_4d(sbase + L::kQ + qs * L::kBoxBytes, &tm_q, bar(L::bQF + qs), 0, cur.h,
+                    cur.qt * kBlockM, cur.b);
         last_q[qs] = i;
+        new_head = cur.advance(p);
       }
       if (!ok) {
         for (int s = 0; s < L::kQStages; ++s)
@@ -154,148 +212,207 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !*abort_flag && cnt > 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN * n_kv, false);
+    setmaxnreg_dec<kSkvRegsIssue>();
+    // The whole warp runs this loop (control values stay warp-uniform); one elected
+    // lane issues each MMA and commit, and the lanes agree on every wait.
+    if (!*abort_flag && cnt > 0) {
+      auto wt = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait_lean(bar_addr, parity, ctl));
+      };
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN * NKV, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
+      // shared-memory descriptors built once; each MMA moves them by a constant offset
+      const SmemDesc dq = SmemDesc::sw128(sbase + L::kQ, 16, 1024);
+      const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
+      const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, L::kBoxBytes, 1024);
       bool issued = false;
-      int kv_ver = -1, cur_bh = -1;
-      // S_b = Q_i K^T into buffer b = i & 1 (waits for Q_i, the buffer and, on a head
-      // change, the new K/V)
-      auto qk = [&](int i) -> bool {
-        const int bh = tile_bh(i);
-        if (bh != cur_bh) {
-          if (!mbar_wait_lean(bar(L::bKVF), (uint32_t)(kv_ver + 1) & 1u, ctl)) return false;
+      int kv_ver = 0;       // K/V loads consumed so far
+      // S = Q_i K^T into buffer i % NB (waits for Q_i and the buffer; `fresh_kv` also
+      // waits for the K/V of a new (batch, head))
+      auto qk = [&](int i, bool fresh_kv) -> bool {
+        if (fresh_kv) {
+          if (!wt(bar(L::bKVF), (uint32_t)kv_ver & 1u)) return false;
           ++kv_ver;
-          cur_bh = bh;
         }
-        const int bf = i & 1;
+        const int bf = i % NB;
         const int qs = i % L::kQStages;
-        if (!mbar_wait_lean(bar(L::bQF + qs), (uint32_t)(i / L::kQStages) & 1u, ctl) ||
-            !mbar_wait_lean(bar(L::bTF + bf), ((uint32_t)(i >> 1) & 1u) ^ 1u, ctl))
+        if (!wt(bar(L::bQF + qs), (uint32_t)(i / L::kQStages) & 1u) ||
+            !wt(bar(L::bTF + bf), ((uint32_t)(i / NB) & 1u) ^ 1u))
           return false;
         tc_fence_after();
-        const uint32_t q_base = sbase + L::kQ + qs * L::kBoxBytes;
+        const uint32_t q_off = (uint32_t)qs * L::kBoxBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + 256 * bf, smem_desc_sw128(q_base + kk * 32, 16, 1024),
-                  smem_desc_sw128(sbase + L::kK + kk * 32, 16, 1024), idesc_qk,
+          umma_ss_elect(tmem + L::kBufCols * bf, dq.at(q_off + kk * 32), dk.at(kk * 32), idesc_qk,
                   kk > 0 ? 1u : 0u);
         issued = true;
-        umma_commit(bar(L::bSF + bf));
-        umma_commit(bar(L::bQE + qs));
+        umma_commit_elect(bar(L::bSF + bf));
+        umma_commit_elect(bar(L::bQE + qs));
         return true;
       };
-      // O_b = P_b V (waits for P_i)
+      // O = P_i V into buffer i % NB (waits for P_i)
       auto pv = [&](int i) -> bool {
-        const int bf = i & 1;
-        if (!mbar_wait_lean(bar(L::bPF + bf), (uint32_t)(i >> 1) & 1u, ctl)) return false;
+        const int bf = i % NB;
+        if (!wt(bar(L::bPF + bf), (uint32_t)(i / NB) & 1u)) return false;
         tc_fence_after();
-        for (int kk = 0; kk < (kBlockN / 16) * n_kv; ++kk)
-          umma_ts(tmem + 256 * bf + L::kColO, tmem + 256 * bf + kk * 8,
-                  smem_desc_sw128(sbase + L::kV + kk * 16 * 128, L::kBoxBytes, 1024), idesc_pv,
-                  kk > 0 ? 1u : 0u);
-        umma_commit(bar(L::bOF + bf));
+        const uint32_t buf = tmem + L::kBufCols * bf;
+#pragma unroll
+        for (int kk = 0; kk < (kBlockN / 16) * NKV; ++kk)
+          umma_ts_elect(buf + L::kColO, buf + kk * 8, dv.at(kk * 16 * 128), idesc_pv, kk > 0 ? 1u : 0u);
+        umma_commit_elect(bar(L::bOF + bf));
         return true;
       };
-      bool ok = qk(0);
+      // QK runs up to kLookahead tiles ahead of PV but never into the next (batch, head)
+      // before every PV of the current one is issued: the K/V buffers are shared.
+      SkvCursor cq;  // tile nq
+      cq.init(t_begin, p);
+      int nq = 0;
+      bool q_fresh = true;    // tile nq starts a (batch, head)
+      bool ok = true;
       for (int i = 0; i < cnt && ok; ++i) {
-        const bool next = i + 1 < cnt;
-        const bool head_change = next && tile_bh(i + 1) != tile_bh(i);
-        if (next && !head_change) ok = qk(i + 1);  // overlap QK(i+1) with softmax(i)
-        if (ok) ok = pv(i);
-        if (ok && head_change) {
-          umma_commit(bar(L::bKVE));  // K/V of the finished head may be overwritten
-          ok = qk(i + 1);
+        while (ok && nq < cnt && nq <= i + L::kLookahead && (!q_fresh || nq == i)) {
+          if (q_fresh && nq > 0) umma_commit_elect(bar(L::bKVE));  // old K/V may be overwritten
+          ok = qk(nq, q_fresh);
+          ++nq;
+          q_fresh = cq.advance(p);
         }
+        if (ok) ok = pv(i);
       }
       if (!ok && issued) {
-        umma_commit(bar(L::bDrain));
+        umma_commit_elect(bar(L::bDrain));
         mbar_wait_drain(bar(L::bDrain), 0, p.timeout_ns);
       }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax + epilogue
-    const int g = (warp >> 2) - 1;  // tiles i with i & 1 == g, TMEM buffer g
+  } else if (warp < 4) {
+    setmaxnreg_dec<kSkvRegsIssue>();  // warps 2-3: idle
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ softmax
+    setmaxnreg_inc<kSkvRegsSoftmax>();
+    const int g = (warp >> 2) - 1;  // tiles i with i & 1 == g
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16) + 256 * g;
+    const uint32_t tlane = tmem + ((uint32_t)(wq * 32) << 16);
     const float sl2 = p.scale_log2;
-    const int nkeys = kBlockN * n_kv;
-    uint8_t* stage = smem + L::kStage + g * L::kBoxBytes;
     bool ok = !*abort_flag;
     for (int i = g; i < cnt && ok; i += 2) {
-      const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-      // the group's four warps agree on every wait, so that all 128 threads leave the
-      // loop together and the named barriers below never wait for a warp that left
-      ok = named_bar_and(1 + g, kBlockM, mbar_wait(bar(L::bSF + g), ph, ctl));
+      const int bf = i % NB;
+      const uint32_t trow = tlane + L::kBufCols * bf;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + bf), (uint32_t)(i / NB) & 1u, ctl));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: exact row max over every valid key
-      float mx = -INFINITY;
-      for (int c = 0; c < nkeys / 32; ++c) {
-        float s[32];
-        tmem_ld32(trow + c * 32, s);
-        tmem_ld_wait();
+      // row sum in two packed accumulators (fp32 pairs)
+      float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
+      const float2 sc2 = make_float2(sl2, sl2);
+      if constexpr (NKV == 1) {
+        // the whole 128-score row in registers: exact max, exponentials, P over the
+        // first 64 columns
+        float s[kBlockN];
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (c * 32 + x < p.kv_valid) mx = fmaxf(mx, s[x]);
-      }
-      const float neg_m = -mx * sl2;
-      // pass 2: exponentials, row sum, P packed over the first nkeys/2 columns (each
-      // chunk's P lands on columns whose scores were already read)
-      float l = 0.0f;
-      for (int c = 0; c < nkeys / 32; ++c) {
-        float s[32];
-        tmem_ld32(trow + c * 32, s);
+        for (int c = 0; c < kBlockN / 32; ++c)
+          tmem_ld32(trow + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
         tmem_ld_wait();
-        uint32_t pk[16];
+        mask_keys<kBlockN / 32>(s, p.kv_valid);
+        const float mx = row_max<kBlockN>(s);
+        const float2 nm2 = make_float2(-mx * sl2, -mx * sl2);
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int k0 = c * 32 + 2 * x;
-          const float p0 = k0 < p.kv_valid ? ex2(fmaf(s[2 * x], sl2, neg_m)) : 0.0f;
-          const float p1 = k0 + 1 < p.kv_valid ? ex2(fmaf(s[2 * x + 1], sl2, neg_m)) : 0.0f;
-          l += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
+          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+          tmem_st16(trow + c * 16, pk);
         }
-        tmem_st16(trow + c * 16, pk);
+      } else {
+        // two key tiles: row max over both (each 128-column half loaded with one wait),
+        // then each half reloaded for its exponentials; P of half t lands on columns
+        // [64t, 64t + 64), whose scores were read before
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int t = 0; t < NKV; ++t) {
+          float s[kBlockN];
+#pragma unroll
+          for (int c = 0; c < kBlockN / 32; ++c)
+            tmem_ld32(trow + t * kBlockN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+          tmem_ld_wait();
+          mask_keys<kBlockN / 32>(s, p.kv_valid - t * kBlockN);
+          mx = fmaxf(mx, row_max<kBlockN>(s));
+        }
+        const float2 nm2 = make_float2(-mx * sl2, -mx * sl2);
+#pragma unroll 1
+        for (int t = 0; t < NKV; ++t) {
+          float s[kBlockN];
+#pragma unroll
+          for (int c = 0; c < kBlockN / 32; ++c)
+            tmem_ld32(trow + t * kBlockN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+          tmem_ld_wait();
+          mask_keys<kBlockN / 32>(s, p.kv_valid - t * kBlockN);
+#pragma unroll
+          for (int c = 0; c < kBlockN / 32; ++c) {
+            uint32_t pk[16];
+            exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+            tmem_st16(trow + t * 64 + c * 16, pk);
+          }
+        }
       }
+      row_sum[bf * kBlockM + row] = (la.x + la.y) + (lb.x + lb.y);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::bPF + g));
-      // epilogue: wait for O, free the TMEM buffer, normalise, stage, TMA store
-      ok = named_bar_and(1 + g, kBlockM, mbar_wait(bar(L::bOF + g), ph, ctl));
+      mbar_arrive(bar(L::bPF + bf));  // P in TMEM and l in shared memory
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    setmaxnreg_dec<kSkvRegsEpi>();
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t tlane = tmem + ((uint32_t)(wq * 32) << 16);
+    const bool leader = wq == 0 && lane == 0;
+    SkvCursor cur;
+    cur.init(t_begin, p);
+    bool ok = !*abort_flag;
+    for (int i = 0; i < cnt && ok; ++i) {
+      const int bf = i % NB;
+      const uint32_t ph = (uint32_t)(i / NB) & 1u;
+      // P_i (and with it l) published, then O_i = P_i V landed; the four warps agree
+      // so that all 128 threads leave the loop together (named barriers follow)
+      bool w = mbar_wait(bar(L::bPF + bf), ph, ctl);
+      w = w && mbar_wait(bar(L::bOF + bf), ph, ctl);
+      ok = named_bar_and(1, kBlockM, w);
       if (!ok) break;
       tc_fence_after();
+      const uint32_t trow = tlane + L::kBufCols * bf;
       float o[D];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c)
         tmem_ld32(trow + L::kColO + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
+      const float inv_l = 1.0f / row_sum[bf * kBlockM + row];
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::bTF + g));  // S/P/O of buffer g may be overwritten now
-      // the previous TMA store from this staging buffer must have read it
-      if (wq == 0 && lane == 0) tma_store_wait_read0();
-      named_bar_sync(1 + g, kBlockM);
-      const float inv_l = 1.0f / l;
+      mbar_arrive(bar(L::bTF + bf));  // S/P/O of this buffer and its l may be reused
+      // the store issued two tiles ago from this staging buffer must have read it
+      const int sb = i & 1;
+      uint8_t* stage = smem + L::kStage + sb * L::kBoxBytes;
+      if (leader) tma_store_wait_read<1>();
+      named_bar_sync(1, kBlockM);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {  // 8 chunks of 16 bytes = 64 bf16
-        const uint32_t w0 = pack_bf16x2(o[8 * u + 0] * inv_l, o[8 * u + 1] * inv_l);
-        const uint32_t w1 = pack_bf16x2(o[8 * u + 2] * inv_l, o[8 * u + 3] * inv_l);
-        const uint32_t w2 = pack_bf16x2(o[8 * u + 4] * inv_l, o[8 * u + 5] * inv_l);
-        const uint32_t w3 = pack_bf16x2(o[8 * u + 6] * inv_l, o[8 * u + 7] * inv_l);
+        const float2 il2 = make_float2(inv_l, inv_l);
+        uint32_t w[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float2 v2 = __fmul2_rn(make_float2(o[8 * u + 2 * x], o[8 * u + 2 * x + 1]), il2);
+          w[x] = pack_bf16x2(v2.x, v2.y);
+        }
         *reinterpret_cast<uint4*>(stage + row * 128 + ((u ^ (row & 7)) << 4)) =
-            make_uint4(w0, w1, w2, w3);
+            make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
-      named_bar_sync(1 + g, kBlockM);
-      if (wq == 0 && lane == 0) {
-        const int bh = tile_bh(i);
-        tma_store_4d(&tm_o, sbase + L::kStage + g * L::kBoxBytes, 0, bh % p.heads,
-                     tile_qt(i) * kBlockM, bh / p.heads);
+      named_bar_sync(1, kBlockM);
+      if (leader) {
+        tma_store_4d(&tm_o, sbase + L::kStage + sb * L::kBoxBytes, 0, cur.h, cur.qt * kBlockM,
+                     cur.b);
         tma_store_commit();
       }
+      cur.advance(p);
     }
-    if (wq == 0 && lane == 0) tma_store_wait_read0();
+    if (leader) tma_store_wait_read<0>();
   }
 
   tc_fence_before();

@@ -88,10 +88,13 @@ bool encode_bshd(const Context& c, CUtensorMap* map, const void* base, int len, 
                                  (cuuint64_t)len * heads * head_dim * 2};
   const cuuint32_t box[4] = {64, 1, (cuuint32_t)ltx::kBlockM, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
+  // L2 fetch granule = one (token, head) row: a 256-byte promotion of a 128-byte row
+  // would also fetch the next head's row, which a head-ordered walk reads much later
+  const CUtensorMapL2promotion promo =
+      head_dim * 2 >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
   CUresult r = c.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_SWIZZLE_128B, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -162,14 +165,22 @@ bool use_short_kv(const FwdParams& p, int head_dim) {
   return head_dim == ltx::kSkvD && p.num_splits == 1 && p.n_kv_tiles <= ltx::kSkvMaxKvTiles;
 }
 
+template <int NKV>
+cudaError_t launch_skv_n(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& to, const FwdParams& p, int grid,
+                         cudaStream_t stream) {
+  ltx::fmha_fwd_skv_sm100<NKV><<<grid, ltx::kSkvThreads, ltx::SkvSmem<NKV>::kAlloc, stream>>>(
+      tq, tk, tv, to, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int num_sms,
                        cudaStream_t stream) {
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
   const int grid = (int)std::min<long long>(total, num_sms);
-  ltx::fmha_fwd_skv_sm100<<<grid, ltx::kSkvThreads, ltx::SkvSmem::kAlloc, stream>>>(tq, tk, tv,
-                                                                                     to, p);
-  return cudaGetLastError();
+  return p.n_kv_tiles == 1 ? launch_skv_n<1>(tq, tk, tv, to, p, grid, stream)
+                           : launch_skv_n<2>(tq, tk, tv, to, p, grid, stream);
 }
 
 template <int D>
@@ -204,8 +215,13 @@ cudaError_t set_smem_limits_pp() {
 }
 
 cudaError_t set_smem_limits_skv() {
-  return cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<false>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, ltx::SkvSmem::kAlloc);
+  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<1>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       ltx::SkvSmem<1>::kAlloc);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<2>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ltx::SkvSmem<2>::kAlloc);
 }
 
 __global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
