@@ -55,12 +55,17 @@ struct FwdParams {
   unsigned long long timeout_ns;
 };
 
-template <int D>
+// kSBuf = 2: S double buffered (QK of tile j+1 overlaps the softmax of tile j), 512
+// TMEM columns, one CTA per SM.  kSBuf = 1: one S buffer, 256 TMEM columns and two K/V
+// stages, so that two CTAs share an SM and interleave their QK -> softmax -> PV chains
+// (head_dim 64 only: shared memory and registers must fit twice).
+template <int D, int kSBuf = 2>
 struct FwdSmem {
+  static_assert(kSBuf == 2 || (kSBuf == 1 && D == 64), "S buffers");
   static constexpr int kBoxes = D / 64;             // 128-byte (64 x bf16) column boxes per row
   static constexpr int kBoxBytes = kBlockM * 128;   // one 128-row x 64-column box
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kStages = (D == 64) ? 3 : 2;
+  static constexpr int kStages = kSBuf == 1 ? 2 : (D == 64) ? 3 : 2;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
@@ -71,8 +76,8 @@ struct FwdSmem {
   static constexpr int bKE = bKF + kStages;
   static constexpr int bVF = bKE + kStages;
   static constexpr int bVE = bVF + kStages;
-  static constexpr int bSF = bVE + kStages;  // 2
-  static constexpr int bPF = bSF + 2;        // 2
+  static constexpr int bSF = bVE + kStages;  // kSBuf
+  static constexpr int bPF = bSF + 2;        // kSBuf
   static constexpr int bOD = bPF + 2;        // O updated by a PV
   static constexpr int bOF = bOD + 1;        // final PV done
   static constexpr int bDrain = bOF + 1;     // abort-path drain
@@ -80,11 +85,12 @@ struct FwdSmem {
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kUsed = kAbort + 4;
-  static constexpr int kAlloc = ((kUsed + 1024 + 1023) / 1024) * 1024 > kMinSmemFor1Cta
-                                    ? ((kUsed + 1024 + 1023) / 1024) * 1024
-                                    : kMinSmemFor1Cta;
-  static constexpr int kColO = 256;
-  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kRaw = ((kUsed + 1024 + 1023) / 1024) * 1024;
+  static constexpr int kAlloc =
+      kSBuf == 1 ? kRaw : (kRaw > kMinSmemFor1Cta ? kRaw : kMinSmemFor1Cta);
+  static constexpr int kColO = 128 * kSBuf;
+  static constexpr uint32_t kTmemCols = kSBuf == 1 ? 256 : 512;
+  static_assert(kSBuf == 2 || 2 * kAlloc <= 227 * 1024, "two CTAs per SM");
 };
 
 // ---------------------------------------------------------------------------
@@ -180,12 +186,12 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
   return true;
 }
 
-template <int D, bool kSplit>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+template <int D, bool kSplit, int kSBuf = 2>
+__global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
     fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams p) {
-  using L = FwdSmem<D>;
+  using L = FwdSmem<D, kSBuf>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -288,8 +294,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
       const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, L::kBoxBytes, 1024);
       auto pv = [&](int t) -> bool {
-        const int sb = t & 1;
-        if (!mbar_wait(bar(L::bPF + sb), (uint32_t)(t >> 1) & 1u, ctl)) return false;
+        const int sb = t % kSBuf;
+        if (!mbar_wait(bar(L::bPF + sb), (uint32_t)(t / kSBuf) & 1u, ctl)) return false;
         const int st = t % L::kStages;
         if (!mbar_wait(bar(L::bVF + st), (uint32_t)(t / L::kStages) & 1u, ctl)) return false;
         tc_fence_after();
@@ -305,11 +311,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         return true;
       };
       for (int j = 0; j < n && ok; ++j) {
+        if (kSBuf == 1 && j >= 1) {
+          // P(j-1) sits in the only S buffer: its PV goes before QK(j) overwrites it
+          ok = pv(j - 1);
+          if (!ok) break;
+        }
         const int st = j % L::kStages;
         ok = mbar_wait(bar(L::bKF + st), (uint32_t)(j / L::kStages) & 1u, ctl);
         if (!ok) break;
         tc_fence_after();
-        const int sb = j & 1;
+        const int sb = j % kSBuf;
         const uint32_t k_off = (uint32_t)st * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -319,7 +330,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         issued = true;
         umma_commit(bar(L::bSF + sb));
         umma_commit(bar(L::bKE + st));
-        if (j >= 1) ok = pv(j - 1);
+        if (kSBuf == 2 && j >= 1) ok = pv(j - 1);
       }
       if (ok) ok = pv(n - 1);
       if (ok) {
@@ -340,26 +351,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float l_run = 0.0f;
     bool ok = !*abort_flag;
     for (int j = 0; j < n && ok; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(j >> 1) & 1u, ctl));
+      const int sb = j % kSBuf;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(j / kSBuf) & 1u, ctl));
       if (!ok) break;
       tc_fence_after();
-      float s[kBlockN];
+      const uint32_t tS = trow + sb * 128;
+      const int lim = p.kv_valid - (kv_begin + j) * kBlockN;  // valid keys in this tile
+      // kSBuf == 2: the whole 128-score row stays in registers.  kSBuf == 1 (two CTAs
+      // per SM, fewer registers): 64-column halves, read twice from TMEM.
+      float s[kSBuf == 2 ? kBlockN : 64];
+      float mx;
+      if constexpr (kSBuf == 2) {
 #pragma unroll
-      for (int c = 0; c < kBlockN / 32; ++c)
-        tmem_ld32(trow + sb * 128 + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-      tmem_ld_wait();
-      const int kv0 = (kv_begin + j) * kBlockN;
-      if (kv0 + kBlockN > p.kv_valid) {
-        const int lim = p.kv_valid - kv0;
+        for (int c = 0; c < kBlockN / 32; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+        tmem_ld_wait();
+        if (lim < kBlockN) {
 #pragma unroll
-        for (int c = 0; c < kBlockN; ++c)
-          if (c >= lim) s[c] = -INFINITY;
+          for (int c = 0; c < kBlockN; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        mx = row_max<kBlockN>(s) * sl2;
+      } else {
+        float m = -INFINITY;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld32(tS + hf * 64, *reinterpret_cast<float(*)[32]>(&s[0]));
+          tmem_ld32(tS + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+          tmem_ld_wait();
+          if (lim < (hf + 1) * 64) mask_keys<2>(s, lim - hf * 64);
+          m = fmaxf(m, row_max<64>(s));
+        }
+        mx = m * sl2;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
-      mx *= sl2;
       if (j == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, mx > m_run + kRescaleThreshold)) {
@@ -385,24 +409,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         l_run *= f;
         m_run = mx;
       }
-      const float neg_m = -m_run;
-      float sum = 0.0f;
+      const float2 nm2 = make_float2(-m_run, -m_run);
+      const float2 sc2 = make_float2(sl2, sl2);
+      float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
+      if constexpr (kSBuf == 2) {
 #pragma unroll
-      for (int c = 0; c < kBlockN / 64; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float p0 = ex2(fmaf(s[c * 64 + 2 * x], sl2, neg_m));
-          const float p1 = ex2(fmaf(s[c * 64 + 2 * x + 1], sl2, neg_m));
-          sum += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
+          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+          tmem_st16(tS + c * 16, pk);
         }
-        tmem_st32(trow + sb * 128 + c * 32, pk);
+      } else {
+        // P of half hf lands on columns [32 hf, 32 hf + 32), read in the first half
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld32(tS + hf * 64, *reinterpret_cast<float(*)[32]>(&s[0]));
+          tmem_ld32(tS + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+          tmem_ld_wait();
+          if (lim < (hf + 1) * 64) mask_keys<2>(s, lim - hf * 64);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t pk[16];
+            exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+            tmem_st16(tS + hf * 32 + c * 16, pk);
+          }
+        }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::bPF + sb));
-      l_run += sum;
+      l_run += (la.x + la.y) + (lb.x + lb.y);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOF), 0, ctl));
     // every softmax thread gets here (all waits are bounded); agree on one outcome so

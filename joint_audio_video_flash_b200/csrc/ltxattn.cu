@@ -23,6 +23,9 @@ using ltx::FwdParams;
 using ltx::FwdSmem;
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+// query sides of at most this many 128-row tiles (head_dim 64, long key side) run the
+// two-CTAs-per-SM variant of the base kernel
+constexpr int kDualMaxQTiles = 1;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -133,12 +136,12 @@ Context* current_context(int* err) {
   return it->second;
 }
 
-template <int D, bool kSplit>
+template <int D, bool kSplit, int kSBuf = 2>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
   dim3 grid(p.n_q_tiles, p.heads, p.batch * p.num_splits);
-  ltx::fmha_fwd_sm100<D, kSplit><<<grid, ltx::kFwdThreads, FwdSmem<D>::kAlloc, stream>>>(
-      tq, tk, tv, to, p);
+  ltx::fmha_fwd_sm100<D, kSplit, kSBuf>
+      <<<grid, ltx::kFwdThreads, FwdSmem<D, kSBuf>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
@@ -191,6 +194,15 @@ cudaError_t launch_combine(const FwdParams& p, void* out, cudaStream_t stream) {
       p.o_part, p.lse_part, reinterpret_cast<__nv_bfloat16*>(out), p.num_splits, p.batch, p.heads,
       p.q_len, p.n_q_tiles * ltx::kBlockM);
   return cudaGetLastError();
+}
+
+cudaError_t set_smem_limits_dual() {
+  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_sm100<64, true, 1>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FwdSmem<64, 1>::kAlloc);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ltx::fmha_fwd_sm100<64, false, 1>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64, 1>::kAlloc);
 }
 
 template <int D>
@@ -281,7 +293,7 @@ int ltxattn_create(void) {
          cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
          set_smem_limits<64>() == cudaSuccess && set_smem_limits<128>() == cudaSuccess &&
          set_smem_limits_pp<64>() == cudaSuccess && set_smem_limits_pp<128>() == cudaSuccess &&
-         set_smem_limits_skv() == cudaSuccess &&
+         set_smem_limits_skv() == cudaSuccess && set_smem_limits_dual() == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
@@ -317,8 +329,12 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   p.timeout_ns = kDefaultTimeoutNs;
 
   const int units = p.n_q_tiles * heads * batch;
+  // head_dim 64 with a long key side and a short query side (v2a): one S buffer per
+  // CTA and two CTAs per SM, so the split planner counts two CTA slots per SM
+  const bool dual = head_dim == 64 && p.n_kv_tiles > ltx::kSkvMaxKvTiles &&
+                    p.n_q_tiles <= kDualMaxQTiles;
   int splits = num_splits > 0 ? std::min(num_splits, p.n_kv_tiles)
-                              : plan_splits(units, p.n_kv_tiles, c->num_sms);
+                              : plan_splits(units, p.n_kv_tiles, (dual ? 2 : 1) * c->num_sms);
   p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
   splits = (p.n_kv_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty part
   if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
@@ -358,6 +374,10 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   cudaError_t e;
   if (use_short_kv(p, head_dim)) {
     e = launch_skv(tq, tk, tv, to, p, c->num_sms, stream);
+  } else if (dual) {
+    e = splits > 1 ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
+                   : launch_fwd<64, false, 1>(tq, tk, tv, to, p, stream);
+    if (e == cudaSuccess && splits > 1) e = launch_combine<64>(p, out, stream);
   } else if (head_dim == 64) {
     e = splits > 1 ? launch_attention<64, true>(tq, tk, tv, to, p, stream)
                    : launch_attention<64, false>(tq, tk, tv, to, p, stream);

@@ -75,6 +75,10 @@ RAGGED = [
     (1, 1, 128, 127, 1025, 1000),
     (1, 3, 128, 200, 256, 129),
     (2, 2, 64, 256, 256, 252),
+    # one query tile over a long key side (two CTAs per SM): split and unsplit
+    (2, 3, 64, 100, 1000, 999),
+    (1, 2, 64, 64, 300, 290),
+    (1, 1, 64, 128, 4096, 4000),
 ]
 
 
@@ -128,15 +132,16 @@ def test_forced_key_splits_two_query_tiles(oracle, d, splits):
     assert_parity(got, ref, f"d={d} splits={splits}")
 
 
-def test_growing_scores_force_rescales(oracle):
+@pytest.mark.parametrize("lq,d,splits", [(130, 128, 0), (100, 64, 1), (100, 64, 2)])
+def test_growing_scores_force_rescales(oracle, lq, d, splits):
     # keys ordered so that the running max grows tile after tile (exercises the O rescale)
-    q, k, v = synth.make_qkv(1, 130, 1024, 2, 128, seed=8)
+    q, k, v = synth.make_qkv(1, lq, 1024, 2, d, seed=8)
     ramp = torch.linspace(0.2, 3.0, 1024).view(1, 1024, 1, 1)
     k = (k.float() * ramp + q[:, :1].float() * ramp * 2).to(torch.bfloat16)
     scale = 0.25
     ref = oracle.attention(q, k, v, scale)
-    got, _ = gpu_run(q, k, v, 1024, scale)
-    assert_parity(got, ref, "ramp")
+    got, _ = gpu_run(q, k, v, 1024, scale, num_splits=splits)
+    assert_parity(got, ref, f"ramp lq={lq} d={d} splits={splits}")
 
 
 def test_large_scores(oracle):
@@ -175,8 +180,9 @@ def test_padding_and_head_slices_are_exact():
     assert torch.equal(base, torch.cat([lo, hi], dim=2))
 
 
-def test_deterministic():
-    q, k, v = synth.make_qkv(1, 384, 3000, 2, 64, seed=12)
+@pytest.mark.parametrize("lq", [384, 100])
+def test_deterministic(lq):
+    q, k, v = synth.make_qkv(1, lq, 3000, 2, 64, seed=12)
     a, _ = gpu_run(q, k, v, 3000, 0.125, num_splits=4)
     b, _ = gpu_run(q, k, v, 3000, 0.125, num_splits=4)
     assert torch.equal(a, b)
