@@ -162,10 +162,13 @@ cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const
                           : launch_fwd<D, kSplit>(tq, tk, tv, to, p, stream);
 }
 
-// Short key side (every valid key in at most two 128-key tiles, head_dim 64):
-// persistent CTAs, one per SM, each walking a contiguous run of query tiles.
-bool use_short_kv(const FwdParams& p, int head_dim) {
-  return head_dim == ltx::kSkvD && p.num_splits == 1 && p.n_kv_tiles <= ltx::kSkvMaxKvTiles;
+// Short key side (every valid key in at most two 128-key tiles, head_dim 64) with more
+// query tiles than SMs: persistent CTAs, one per SM, each walking a contiguous run of
+// query tiles.  With at most one tile per SM (audio self-attention) the one-tile CTAs of
+// the base kernels start faster.
+bool use_short_kv(const FwdParams& p, int head_dim, int num_sms) {
+  return head_dim == ltx::kSkvD && p.num_splits == 1 && p.n_kv_tiles <= ltx::kSkvMaxKvTiles &&
+         (long long)p.batch * p.heads * p.n_q_tiles > num_sms;
 }
 
 template <int NKV>
@@ -372,7 +375,7 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   }
 
   cudaError_t e;
-  if (use_short_kv(p, head_dim)) {
+  if (use_short_kv(p, head_dim, c->num_sms)) {
     e = launch_skv(tq, tk, tv, to, p, c->num_sms, stream);
   } else if (dual) {
     e = splits > 1 ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
