@@ -174,22 +174,28 @@ def cpu_baseline(calls, target_s: float, seed: int = 0):
 
 
 # --------------------------------------------------------------------------- dist
-def dist_setup(n_gpus: int):
-    import torch
+def dist_setup(n_gpus: int, backend: str = "nccl", timeout_s: float = 120.0):
+    """Process group for N replicas (one process per GPU; torchrun's env variables).
+
+    Only the barrier and the max-over-ranks timing use it: every (batch, head) of every call
+    is independent, so there is no data-path collective.  `backend` "gloo" runs the same
+    host logic on CPU processes (tests).
+    """
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != n_gpus and world > 1:
         raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if backend == "nccl":
+        import torch
+        torch.cuda.set_device(local if world > 1 else 0)
     if world > 1:
         import datetime
 
+        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return world, rank, local
 
 
@@ -200,13 +206,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest x over all ranks (the job's time is its slowest replica's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(step_flops: float, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the max-over-ranks device time."""
+    return step_flops * steps * world / (total_ms * 1e-3) / 1e12
 
 
 # --------------------------------------------------------------------------- main arms
@@ -316,7 +329,7 @@ def run_ltxattn(args):
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
     step_flops = sum(c.flops for c in calls)
-    value = step_flops * args.steps * world / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(step_flops, args.steps, world, total_ms)
 
     call_us = []
     for i, c in enumerate(calls):
@@ -355,7 +368,7 @@ def run_ltxattn(args):
     barrier(world)
     ltxattn.check()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(step_flops, e2e_steps, world, e2e_ms)
 
     peaks, peak_src = load_peaks()
     # dominant kernel: the video self-attention (tensor-core bound).  Its denominator is
