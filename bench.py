@@ -337,22 +337,46 @@ def run_ltxattn(args):
         call_us.append(ts)
     launches_per_step = sum(1 if sp == 1 else 2 for sp in splits)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Every step uploads all
+    # inputs from pinned host memory and downloads every output; uploads run on one copy
+    # stream and downloads on another (PCIe is full duplex), each call's kernel waits for
+    # its own upload, and an upload into a device buffer waits for the previous step's
+    # kernel that read it.
     pinned = [tuple(t.pin_memory() for t in trip) for trip in host]
     host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
     h2d = sum(t.numel() * t.element_size() for trip in pinned for t in trip)
     d2h = sum(o.numel() * o.element_size() for o in host_out)
     e2e_steps = max(1, min(args.steps, 5))
+    up_stream = torch.cuda.Stream(device=dev)
+    down_stream = torch.cuda.Stream(device=dev)
+    consumed = [None] * len(calls)   # event: call i's kernel of the previous step finished
+    drained = [None] * len(calls)    # event: call i's output of the previous step downloaded
 
     def e2e_step():
         for i, c in enumerate(calls):
             dq, dk, dv = dev_in[i]
             hq, hk, hv = pinned[i]
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
+            with torch.cuda.stream(up_stream):
+                if consumed[i] is not None:
+                    up_stream.wait_event(consumed[i])
+                dq.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                uploaded = torch.cuda.Event()
+                uploaded.record(up_stream)
+            stream.wait_event(uploaded)
+            if drained[i] is not None:
+                stream.wait_event(drained[i])
             ltxattn.forward(dq, dk, dv, outs[i], kv_valid_len=c.kv_valid_len, scale=c.scale)
-            host_out[i].copy_(outs[i], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(stream)
+            consumed[i] = done
+            with torch.cuda.stream(down_stream):
+                down_stream.wait_event(done)
+                host_out[i].copy_(outs[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(down_stream)
+                drained[i] = ev
 
     e2e_step()
     torch.cuda.synchronize()
@@ -361,8 +385,12 @@ def run_ltxattn(args):
     barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)
+    up_stream.wait_event(e0)  # no copy of the timed steps starts before the start event
     for _ in range(e2e_steps):
         e2e_step()
+    # the timed region ends when the last download has landed
+    for ev in drained:
+        stream.wait_event(ev)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)

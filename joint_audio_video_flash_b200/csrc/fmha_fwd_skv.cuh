@@ -35,6 +35,9 @@ constexpr int kSkvRegsLaunch = 128;  // 65536 / 512
 constexpr int kSkvRegsIssue = 56;    // warps 0-3
 constexpr int kSkvRegsEpi = 104;     // warps 12-15
 constexpr int kSkvRegsSoftmax = 176; // warps 4-11
+// every kSkvExp2FmaEvery-th pair of exponentials of the two-key-tile path runs on the FMA
+// pipe (0 = none)
+constexpr int kSkvExp2FmaEvery = 0;
 static_assert(128 * kSkvRegsIssue + 128 * kSkvRegsEpi + 256 * kSkvRegsSoftmax <=
                   kSkvThreads * kSkvRegsLaunch,
               "register split exceeds the launch allocation");
@@ -321,35 +324,60 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
           tmem_st16(trow + c * 16, pk);
         }
       } else {
-        // two key tiles: row max over both (each 128-column half loaded with one wait),
-        // then each half reloaded for its exponentials; P of half t lands on columns
-        // [64t, 64t + 64), whose scores were read before
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int t = 0; t < NKV; ++t) {
-          float s[kBlockN];
+        // Two key tiles.  The softmax needs a stabiliser close to the row max, not the
+        // max itself: the first tile's max m_a stabilises its exponentials at once; the
+        // second tile reuses m_a unless its max exceeds m_a by more than 2^6 (then its
+        // probabilities could overflow bf16's useful range), in which case this warp
+        // redoes the row with the exact max over both tiles.
+        float s[kBlockN];
 #pragma unroll
-          for (int c = 0; c < kBlockN / 32; ++c)
-            tmem_ld32(trow + t * kBlockN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-          tmem_ld_wait();
-          mask_keys<kBlockN / 32>(s, p.kv_valid - t * kBlockN);
-          mx = fmaxf(mx, row_max<kBlockN>(s));
+        for (int c = 0; c < kBlockN / 32; ++c)
+          tmem_ld32(trow + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+        tmem_ld_wait();
+        mask_keys<kBlockN / 32>(s, p.kv_valid);
+        float m = row_max<kBlockN>(s);
+        float2 nm2 = make_float2(-m * sl2, -m * sl2);
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
+          exp2_pack16<kSkvExp2FmaEvery>(&s[c * 32], sc2, nm2, la, lb, pk);
+          tmem_st16(trow + c * 16, pk);
         }
-        const float2 nm2 = make_float2(-mx * sl2, -mx * sl2);
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c)
+          tmem_ld32(trow + kBlockN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+        tmem_ld_wait();
+        mask_keys<kBlockN / 32>(s, p.kv_valid - kBlockN);
+        const float mb = row_max<kBlockN>(s);
+        if (__any_sync(0xffffffffu, (mb - m) * sl2 > 64.0f)) {
+          // rare (a row whose second tile outgrows the first by more than 2^64): raise
+          // the stabiliser to the larger max; the first tile's P, already in TMEM, and its
+          // partial sums scale by f = 2^((m - m_new) * scale_log2) <= 1 (f = 1 on the
+          // lanes whose max did not move; tcgen05.ld/st are warp-collective)
+          const float mn = fmaxf(m, mb);
+          const float f = ex2((m - mn) * sl2);
+          m = mn;
+          nm2 = make_float2(-m * sl2, -m * sl2);
+          la = make_float2(la.x * f, la.y * f);
+          lb = make_float2(lb.x * f, lb.y * f);
+          tmem_st_wait();
 #pragma unroll 1
-        for (int t = 0; t < NKV; ++t) {
-          float s[kBlockN];
+          for (int c = 0; c < 4; ++c) {  // 64 columns of packed bf16 pairs, 16 at a time
+            uint32_t u[16];
+            tmem_ld16(trow + c * 16, u);
+            tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < kBlockN / 32; ++c)
-            tmem_ld32(trow + t * kBlockN + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-          tmem_ld_wait();
-          mask_keys<kBlockN / 32>(s, p.kv_valid - t * kBlockN);
-#pragma unroll
-          for (int c = 0; c < kBlockN / 32; ++c) {
-            uint32_t pk[16];
-            exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
-            tmem_st16(trow + t * 64 + c * 16, pk);
+            for (int x = 0; x < 16; ++x)
+              u[x] = pack_bf16x2(__uint_as_float(u[x] << 16) * f,
+                                 __uint_as_float(u[x] & 0xffff0000u) * f);
+            tmem_st16(trow + c * 16, u);
           }
+        }
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
+          exp2_pack16<kSkvExp2FmaEvery>(&s[c * 32], sc2, nm2, la, lb, pk);
+          tmem_st16(trow + 64 + c * 16, pk);
         }
       }
       row_sum[bf * kBlockM + row] = (la.x + la.y) + (lb.x + lb.y);

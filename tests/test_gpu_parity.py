@@ -111,6 +111,22 @@ def test_short_kv_persistent_walks(oracle, shape):
     assert_parity(got, oracle.attention(q, k, v, 0.125, kv_valid_len=valid), str(shape))
 
 
+@pytest.mark.parametrize("gain", [0.5, 4.0])
+def test_short_kv_second_tile_outgrows_first(oracle, gain):
+    # two key tiles; the second tile's keys point along query 0, so rows' scores there
+    # exceed the first tile's by a little (gain 0.5: large probabilities stored against
+    # the first tile's max) or by far more than 2^64 (gain 4: the first tile's P is
+    # rescaled to the larger max)
+    b, h, lq, lkv, valid = 1, 40, 512, 256, 252
+    q, k, v = synth.make_qkv(b, lq, lkv, h, 64, seed=41, kv_valid=valid)
+    k = k.float()
+    k[:, 128:valid] = k[:, 128:valid] * 0.25 + q[:, :1].float() * gain
+    k = k.to(torch.bfloat16)
+    got, used = gpu_run(q, k, v, valid, 1.0)
+    assert used == 1
+    assert_parity(got, oracle.attention(q, k, v, 1.0, kv_valid_len=valid), f"gain={gain}")
+
+
 @pytest.mark.parametrize("splits", [1, 2, 3, 5, 16, 40])
 def test_forced_key_splits(oracle, splits):
     # v2a-like: few query rows, many keys; 2000 valid keys = 16 tiles (ragged last one)
