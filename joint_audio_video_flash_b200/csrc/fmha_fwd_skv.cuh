@@ -1,7 +1,8 @@
-// fmha_fwd_skv.cuh -- attention forward for a short key side (at most 256 keys) and
-// head_dim 64 on sm_100a: a2v (video queries over the padded audio keys/values) and
-// audio self-attention of an LTX-2 block ("LTX-2: replicate audio stream across
-// Ulysses ranks by default", Description).  Same operation, layout and key mask as
+// fmha_fwd_skv.cuh -- attention forward for a short key side (at most 256 keys) on
+// sm_100a: a2v (video queries over the padded audio keys/values) of an LTX-2 block
+// ("LTX-2: replicate audio stream across Ulysses ranks by default", Description), at
+// head_dim 64, and the streams' queries over a padded text context at head_dim 64 or
+// 128.  Same operation, layout and key mask as
 // fmha_fwd.cuh.  With every key in one S tile the softmax max is exact, so there is
 // no online rescale.  The work is bound by HBM (reading Q, writing O) and by the
 // exponentials, so the design keeps both busy at once:
@@ -17,10 +18,12 @@
 //   - warps 12-15: the epilogue warpgroup takes every tile in order: waits for O,
 //     divides by l, rounds to bf16, stages the tile (two staging buffers) and
 //     issues its TMA store.
-// TMEM (512 columns) holds NB = 4 / NKV buffers of 128*NKV columns; tile i uses buffer
-// i % NB.  In a buffer: S over all 128*NKV columns, P packed as bf16 pairs over the
-// first 64*NKV columns (written after the scores it replaces were read), O (64 fp32
-// columns) right after P, over scores already read.
+// TMEM (512 columns) holds NB buffers (4 / NKV at head_dim 64, 2 at 128); tile i uses
+// buffer i % NB.  In a buffer: S over the first 128*NKV columns, P packed as bf16 pairs
+// over the first 64*NKV columns (written after the scores it replaces were read), O (D
+// fp32 columns) right after P, over scores already read.  K and V are stored box-major
+// ([64-column box][key tile]), so that QK over two key tiles (N = 256) and PV over 256
+// keys see one contiguous row range per box.
 // Registers (setmaxnreg): producer/MMA warpgroup 56, epilogue 104, softmax 176.
 #pragma once
 
@@ -29,7 +32,6 @@
 namespace ltx {
 
 constexpr int kSkvThreads = 512;
-constexpr int kSkvD = 64;
 constexpr int kSkvMaxKvTiles = 2;
 constexpr int kSkvRegsLaunch = 128;  // 65536 / 512
 constexpr int kSkvRegsIssue = 56;    // warps 0-3
@@ -42,22 +44,27 @@ static_assert(128 * kSkvRegsIssue + 128 * kSkvRegsEpi + 256 * kSkvRegsSoftmax <=
                   kSkvThreads * kSkvRegsLaunch,
               "register split exceeds the launch allocation");
 
-template <int NKV>
+template <int D, int NKV>
 struct SkvSmem {
   static_assert(NKV == 1 || NKV == 2, "one or two 128-key tiles");
+  static_assert(D == 64 || D == 128, "head_dim");
+  static constexpr int kBoxes = D / 64;            // 64-column (128-byte) boxes per row
   static constexpr int kBoxBytes = kBlockM * 128;  // 128 rows x 64 bf16
-  static constexpr int kQStages = NKV == 1 ? 8 : 6;
-  static constexpr int kNB = 4 / NKV;                   // TMEM buffers
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kQStages = D == 64 ? (NKV == 1 ? 8 : 6) : (NKV == 1 ? 3 : 2);
+  static constexpr int kStaging = D == 64 ? 2 : 1;      // output staging tiles
+  static constexpr uint32_t kBufCols = D == 64 ? 128u * NKV : 256u;  // columns per buffer
+  static constexpr int kNB = (int)(512u / kBufCols);    // TMEM buffers
   // QK runs this many tiles ahead of PV; QK(i + kLookahead) reuses the buffer of tile
   // i + kLookahead - kNB, whose epilogue needs PV(i + kLookahead - kNB) issued earlier
   static constexpr int kLookahead = kNB - 1 < 2 ? kNB - 1 : 2;
-  static constexpr uint32_t kBufCols = 128u * NKV;      // columns per buffer
   static constexpr uint32_t kColO = 64u * NKV;          // O within a buffer (after P)
-  static constexpr int kK = 0;                          // NKV key tiles
-  static constexpr int kV = kK + NKV * kBoxBytes;
-  static constexpr int kQ = kV + NKV * kBoxBytes;       // Q ring
-  static constexpr int kStage = kQ + kQStages * kBoxBytes;  // 2 output staging buffers
-  static constexpr int kRowSum = kStage + 2 * kBoxBytes;    // l per buffer and row (fp32)
+  static_assert(kColO + D <= kBufCols, "O fits its buffer");
+  static constexpr int kK = 0;                          // [box][key tile]
+  static constexpr int kV = kK + NKV * kTileBytes;
+  static constexpr int kQ = kV + NKV * kTileBytes;      // Q ring
+  static constexpr int kStage = kQ + kQStages * kTileBytes;       // output staging
+  static constexpr int kRowSum = kStage + kStaging * kTileBytes;  // l per buffer and row
   static constexpr int kBar = kRowSum + kNB * kBlockM * 4;
   static constexpr int bKVF = 0;
   static constexpr int bKVE = 1;
@@ -112,14 +119,13 @@ __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
 }
 
-template <int NKV>
+template <int D, int NKV>
 __global__ void __launch_bounds__(kSkvThreads, 1)
     fmha_fwd_skv_sm100(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
-  using L = SkvSmem<NKV>;
-  constexpr int D = kSkvD;
+  using L = SkvSmem<D, NKV>;
   constexpr int NB = L::kNB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -185,22 +191,27 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
         if (new_head) {
           if (kv_loads > 0) ok = mbar_wait_lean(bar(L::bKVE), (uint32_t)(kv_loads - 1) & 1u, ctl);
           if (!ok) break;
-          mbar_arrive_expect_tx(bar(L::bKVF), 2 * NKV * L::kBoxBytes);
+          mbar_arrive_expect_tx(bar(L::bKVF), 2 * NKV * L::kTileBytes);
 #pragma unroll
-          for (int t = 0; t < NKV; ++t) {
-            tma_load_4d(sbase + L::kK + t * L::kBoxBytes, &tm_k, bar(L::bKVF), 0, cur.h,
-                        t * kBlockN, cur.b);
-            tma_load_4d(sbase + L::kV + t * L::kBoxBytes, &tm_v, bar(L::bKVF), 0, cur.h,
-                        t * kBlockN, cur.b);
-          }
+          for (int bx = 0; bx < L::kBoxes; ++bx)
+#pragma unroll
+            for (int t = 0; t < NKV; ++t) {
+              const uint32_t off = (uint32_t)(bx * NKV + t) * L::kBoxBytes;
+              tma_load_4d(sbase + L::kK + off, &tm_k, bar(L::bKVF), bx * 64, cur.h,
+                          t * kBlockN, cur.b);
+              tma_load_4d(sbase + L::kV + off, &tm_v, bar(L::bKVF), bx * 64, cur.h,
+                          t * kBlockN, cur.b);
+            }
           ++kv_loads;
         }
         const int qs = i % L::kQStages;
         ok = mbar_wait_lean(bar(L::bQE + qs), ((uint32_t)(i / L::kQStages) & 1u) ^ 1u, ctl);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::bQF + qs), L::kBoxBytes);
-        tma_load_4d(sbase + L::kQ + qs * L::kBoxBytes, &tm_q, bar(L::bQF + qs), 0, cur.h,
-                    cur.qt * kBlockM, cur.b);
+        mbar_arrive_expect_tx(bar(L::bQF + qs), L::kTileBytes);
+#pragma unroll
+        for (int bx = 0; bx < L::kBoxes; ++bx)
+          tma_load_4d(sbase + L::kQ + qs * L::kTileBytes + bx * L::kBoxBytes, &tm_q,
+                      bar(L::bQF + qs), bx * 64, cur.h, cur.qt * kBlockM, cur.b);
         last_q[qs] = i;
         new_head = cur.advance(p);
       }
@@ -227,7 +238,8 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       // shared-memory descriptors built once; each MMA moves them by a constant offset
       const SmemDesc dq = SmemDesc::sw128(sbase + L::kQ, 16, 1024);
       const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
-      const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, L::kBoxBytes, 1024);
+      // V is MN-major: its leading byte offset steps from one 64-column box to the next
+      const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, NKV * L::kBoxBytes, 1024);
       bool issued = false;
       int kv_ver = 0;       // K/V loads consumed so far
       // S = Q_i K^T into buffer i % NB (waits for Q_i and the buffer; `fresh_kv` also
@@ -243,11 +255,15 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
             !wt(bar(L::bTF + bf), ((uint32_t)(i / NB) & 1u) ^ 1u))
           return false;
         tc_fence_after();
-        const uint32_t q_off = (uint32_t)qs * L::kBoxBytes;
+        const uint32_t q_off = (uint32_t)qs * L::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss_elect(tmem + L::kBufCols * bf, dq.at(q_off + kk * 32), dk.at(kk * 32), idesc_qk,
-                  kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // 16 head-dim columns: box kk / 4, 32-byte step kk % 4 within the box
+          const uint32_t in_box = (kk & 3) * 32;
+          umma_ss_elect(tmem + L::kBufCols * bf, dq.at(q_off + (kk >> 2) * L::kBoxBytes + in_box),
+                        dk.at((kk >> 2) * NKV * L::kBoxBytes + in_box), idesc_qk,
+                        kk > 0 ? 1u : 0u);
+        }
         issued = true;
         umma_commit_elect(bar(L::bSF + bf));
         umma_commit_elect(bar(L::bQE + qs));
@@ -406,36 +422,42 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t trow = tlane + L::kBufCols * bf;
-      float o[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c)
-        tmem_ld32(trow + L::kColO + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
       const float inv_l = 1.0f / row_sum[bf * kBlockM + row];
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::bTF + bf));  // S/P/O of this buffer and its l may be reused
-      // the store issued two tiles ago from this staging buffer must have read it
-      const int sb = i & 1;
-      uint8_t* stage = smem + L::kStage + sb * L::kBoxBytes;
-      if (leader) tma_store_wait_read<1>();
+      // the store issued kStaging tiles ago from this staging buffer must have read it
+      const int sb = L::kStaging == 2 ? (i & 1) : 0;
+      uint8_t* stage = smem + L::kStage + sb * L::kTileBytes;
+      if (leader) tma_store_wait_read<L::kStaging - 1>();
       named_bar_sync(1, kBlockM);
+      const float2 il2 = make_float2(inv_l, inv_l);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // 8 chunks of 16 bytes = 64 bf16
-        const float2 il2 = make_float2(inv_l, inv_l);
-        uint32_t w[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float2 v2 = __fmul2_rn(make_float2(o[8 * u + 2 * x], o[8 * u + 2 * x + 1]), il2);
-          w[x] = pack_bf16x2(v2.x, v2.y);
+      for (int bx = 0; bx < L::kBoxes; ++bx) {  // 64 output columns per box
+        float o[64];
+        tmem_ld32(trow + L::kColO + bx * 64, *reinterpret_cast<float(*)[32]>(&o[0]));
+        tmem_ld32(trow + L::kColO + bx * 64 + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+        tmem_ld_wait();
+        if (bx == L::kBoxes - 1) {
+          tc_fence_before();
+          mbar_arrive(bar(L::bTF + bf));  // S/P/O of this buffer and its l may be reused
         }
-        *reinterpret_cast<uint4*>(stage + row * 128 + ((u ^ (row & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {  // 8 chunks of 16 bytes = 64 bf16
+          uint32_t w[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float2 v2 = __fmul2_rn(make_float2(o[8 * u + 2 * x], o[8 * u + 2 * x + 1]), il2);
+            w[x] = pack_bf16x2(v2.x, v2.y);
+          }
+          *reinterpret_cast<uint4*>(stage + bx * L::kBoxBytes + row * 128 +
+                                    ((u ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
       }
       fence_proxy_async_smem();
       named_bar_sync(1, kBlockM);
       if (leader) {
-        tma_store_4d(&tm_o, sbase + L::kStage + sb * L::kBoxBytes, 0, cur.h, cur.qt * kBlockM,
-                     cur.b);
+#pragma unroll
+        for (int bx = 0; bx < L::kBoxes; ++bx)
+          tma_store_4d(&tm_o, sbase + L::kStage + sb * L::kTileBytes + bx * L::kBoxBytes,
+                       bx * 64, cur.h, cur.qt * kBlockM, cur.b);
         tma_store_commit();
       }
       cur.advance(p);

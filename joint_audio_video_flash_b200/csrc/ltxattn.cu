@@ -1,7 +1,8 @@
 // ltxattn.cu -- host side of the C ABI declared in include/ltxattn.h: argument
 // validation, per-device context, TMA tensor maps, key-range split planning,
 // workspace and kernel launches.  No CPU compute path exists: every step of the
-// attention runs in the kernels of fmha_fwd.cuh and combine.cuh.
+// attention runs in the kernels of fmha_fwd.cuh, fmha_fwd_pp.cuh, fmha_fwd_skv.cuh and
+// combine.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -162,31 +163,34 @@ cudaError_t launch_attention(const CUtensorMap& tq, const CUtensorMap& tk, const
                           : launch_fwd<D, kSplit>(tq, tk, tv, to, p, stream);
 }
 
-// Short key side (every valid key in at most two 128-key tiles, head_dim 64) with more
-// query tiles than SMs: persistent CTAs, one per SM, each walking a contiguous run of
-// query tiles.  With at most one tile per SM (audio self-attention) the one-tile CTAs of
-// the base kernels start faster.
-bool use_short_kv(const FwdParams& p, int head_dim, int num_sms) {
-  return head_dim == ltx::kSkvD && p.num_splits == 1 && p.n_kv_tiles <= ltx::kSkvMaxKvTiles &&
+// Short key side (every valid key in at most two 128-key tiles) with more query tiles
+// than SMs: persistent CTAs, one per SM, each walking a contiguous run of query tiles.
+// With at most one tile per SM (audio self-attention) the one-tile CTAs of the base
+// kernels start faster.
+bool use_short_kv(const FwdParams& p, int num_sms) {
+  return p.num_splits == 1 && p.n_kv_tiles <= ltx::kSkvMaxKvTiles &&
          (long long)p.batch * p.heads * p.n_q_tiles > num_sms;
 }
 
-template <int NKV>
+template <int D, int NKV>
 cudaError_t launch_skv_n(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& to, const FwdParams& p, int grid,
                          cudaStream_t stream) {
-  ltx::fmha_fwd_skv_sm100<NKV><<<grid, ltx::kSkvThreads, ltx::SkvSmem<NKV>::kAlloc, stream>>>(
-      tq, tk, tv, to, p);
+  ltx::fmha_fwd_skv_sm100<D, NKV>
+      <<<grid, ltx::kSkvThreads, ltx::SkvSmem<D, NKV>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, const FwdParams& p, int num_sms,
+                       const CUtensorMap& to, const FwdParams& p, int head_dim, int num_sms,
                        cudaStream_t stream) {
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
   const int grid = (int)std::min<long long>(total, num_sms);
-  return p.n_kv_tiles == 1 ? launch_skv_n<1>(tq, tk, tv, to, p, grid, stream)
-                           : launch_skv_n<2>(tq, tk, tv, to, p, grid, stream);
+  if (head_dim == 64)
+    return p.n_kv_tiles == 1 ? launch_skv_n<64, 1>(tq, tk, tv, to, p, grid, stream)
+                             : launch_skv_n<64, 2>(tq, tk, tv, to, p, grid, stream);
+  return p.n_kv_tiles == 1 ? launch_skv_n<128, 1>(tq, tk, tv, to, p, grid, stream)
+                           : launch_skv_n<128, 2>(tq, tk, tv, to, p, grid, stream);
 }
 
 template <int D>
@@ -229,14 +233,19 @@ cudaError_t set_smem_limits_pp() {
                               ltx::PPSmem<D>::kAlloc);
 }
 
-cudaError_t set_smem_limits_skv() {
-  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<1>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       ltx::SkvSmem<1>::kAlloc);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<2>,
+template <int D, int NKV>
+cudaError_t set_smem_limit_skv() {
+  return cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<D, NKV>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              ltx::SkvSmem<2>::kAlloc);
+                              ltx::SkvSmem<D, NKV>::kAlloc);
+}
+
+cudaError_t set_smem_limits_skv() {
+  cudaError_t e = set_smem_limit_skv<64, 1>();
+  if (e == cudaSuccess) e = set_smem_limit_skv<64, 2>();
+  if (e == cudaSuccess) e = set_smem_limit_skv<128, 1>();
+  if (e == cudaSuccess) e = set_smem_limit_skv<128, 2>();
+  return e;
 }
 
 __global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
@@ -375,8 +384,8 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   }
 
   cudaError_t e;
-  if (use_short_kv(p, head_dim, c->num_sms)) {
-    e = launch_skv(tq, tk, tv, to, p, c->num_sms, stream);
+  if (use_short_kv(p, c->num_sms)) {
+    e = launch_skv(tq, tk, tv, to, p, head_dim, c->num_sms, stream);
   } else if (dual) {
     e = splits > 1 ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
                    : launch_fwd<64, false, 1>(tq, tk, tv, to, p, stream);

@@ -20,7 +20,7 @@ from dataclasses import dataclass
 
 @dataclass(frozen=True)
 class Call:
-    name: str            # video_self | audio_self | v2a | a2v
+    name: str            # video_self | audio_self | v2a | a2v | v2t | a2t
     batch: int
     q_len: int
     kv_len: int
@@ -62,7 +62,7 @@ def _audio_stream(cfg: int, batch: int, video: int, audio_pad: int, audio_valid:
 
 
 def configs() -> dict:
-    """The five workloads, keyed by a short name; values are (description, [Call, ...])."""
+    """The workloads, keyed by a short name; values are (description, [Call, ...])."""
     tiny = [
         Call("video_self", 1, 256, 256, 256, 2, 64, 256, _seed(1, 0)),
         Call("audio_self", 1, 8, 8, 8, 2, 64, 8, _seed(1, 1)),
@@ -85,6 +85,12 @@ def configs() -> dict:
                       "(32x128, 201 MB of inputs) + a2v and v2a at the 768x1280x121 block size",
                       [Call("video_self", 1, 8192, 8192, 8192, 32, 128, 8192, _seed(6, 0))]
                       + _audio_stream(6, 2, 15360, 128, 126, 1)[1:]),
+        "text_xattn": ("text cross-attention at 768x1280x121, B2: video queries 15360 (32x128) "
+                       "and audio queries 126->128 (32x64) over a text context padded to 1024 "
+                       "tokens with 256 valid (the context length is a reading: the pages "
+                       "give none)",
+                       [Call("v2t", 2, 15360, 1024, 256, 32, 128, 15360, _seed(7, 0)),
+                        Call("a2t", 2, 128, 1024, 256, 32, 64, 126, _seed(7, 1))]),
         "longclip": ("long clip 1280x704x241 (27280 video tokens), audio 252->256 masked, B2: "
                      "video self (32x128) + audio self + v2a + a2v (32x64)",
                      [Call("video_self", 2, 27280, 27280, 27280, 32, 128, 27280, _seed(5, 0))]

@@ -94,37 +94,44 @@ def test_ragged_shapes_full(oracle, shape):
 SHORT_KV_WALKS = [
     # more (batch, head, query tile) units than SMs: persistent CTAs cross head
     # boundaries, reloading K/V; one query tile per head makes every tile a new head
-    (4, 64, 128, 128, 126),
-    (3, 50, 200, 256, 252),
+    (4, 64, 128, 128, 126, 64),
+    (3, 50, 200, 256, 252, 64),
     # eight query tiles per head, two key tiles with the second holding one valid key
-    (2, 16, 1000, 256, 129),
-    (1, 40, 2000, 300, 256),
+    (2, 16, 1000, 256, 129, 64),
+    (1, 40, 2000, 300, 256, 64),
+    # head_dim 128 (two 64-column boxes per row): one and two key tiles, and a padded
+    # text-like key side (1024 rows, 256 valid)
+    (1, 64, 300, 128, 100, 128),
+    (2, 32, 512, 256, 252, 128),
+    (2, 20, 1000, 1024, 256, 128),
 ]
 
 
-@pytest.mark.parametrize("shape", SHORT_KV_WALKS, ids=lambda s: "b{}h{}_q{}_kv{}v{}".format(*s))
+@pytest.mark.parametrize("shape", SHORT_KV_WALKS,
+                         ids=lambda s: "b{}h{}_q{}_kv{}v{}_d{}".format(*s))
 def test_short_kv_persistent_walks(oracle, shape):
-    b, h, lq, lkv, valid = shape
-    q, k, v = synth.make_qkv(b, lq, lkv, h, 64, seed=31 + lq + h, kv_valid=valid)
-    got, used = gpu_run(q, k, v, valid, 0.125)
+    b, h, lq, lkv, valid, d = shape
+    q, k, v = synth.make_qkv(b, lq, lkv, h, d, seed=31 + lq + h, kv_valid=valid)
+    scale = 1.0 / np.sqrt(d)
+    got, used = gpu_run(q, k, v, valid, scale)
     assert used == 1
-    assert_parity(got, oracle.attention(q, k, v, 0.125, kv_valid_len=valid), str(shape))
+    assert_parity(got, oracle.attention(q, k, v, scale, kv_valid_len=valid), str(shape))
 
 
-@pytest.mark.parametrize("gain", [0.5, 4.0])
-def test_short_kv_second_tile_outgrows_first(oracle, gain):
+@pytest.mark.parametrize("gain,d", [(0.5, 64), (4.0, 64), (4.0, 128)])
+def test_short_kv_second_tile_outgrows_first(oracle, gain, d):
     # two key tiles; the second tile's keys point along query 0, so rows' scores there
     # exceed the first tile's by a little (gain 0.5: large probabilities stored against
     # the first tile's max) or by far more than 2^64 (gain 4: the first tile's P is
     # rescaled to the larger max)
     b, h, lq, lkv, valid = 1, 40, 512, 256, 252
-    q, k, v = synth.make_qkv(b, lq, lkv, h, 64, seed=41, kv_valid=valid)
+    q, k, v = synth.make_qkv(b, lq, lkv, h, d, seed=41, kv_valid=valid)
     k = k.float()
     k[:, 128:valid] = k[:, 128:valid] * 0.25 + q[:, :1].float() * gain
     k = k.to(torch.bfloat16)
     got, used = gpu_run(q, k, v, valid, 1.0)
     assert used == 1
-    assert_parity(got, oracle.attention(q, k, v, 1.0, kv_valid_len=valid), f"gain={gain}")
+    assert_parity(got, oracle.attention(q, k, v, 1.0, kv_valid_len=valid), f"gain={gain} d={d}")
 
 
 @pytest.mark.parametrize("splits", [1, 2, 3, 5, 16, 40])
@@ -238,6 +245,20 @@ def test_block768_sampled(oracle):
     _, calls = workloads.configs()["block768"]
     for c in calls:
         _sampled(oracle, c, per_head=4, full_heads=((1, 5),), tail_block=64)
+
+
+def test_text_cross_attention(oracle):
+    # video and audio queries over a padded text context (keys >= 256 masked)
+    _, calls = workloads.configs()["text_xattn"]
+    for c in calls:
+        if c.q_len <= 256:
+            q, k, v = synth.make_qkv(c.batch, c.q_len, c.kv_len, c.heads, c.head_dim, c.seed,
+                                     q_valid=c.q_valid, kv_valid=c.kv_valid_len)
+            got, _ = gpu_run(q, k, v, c.kv_valid_len, c.scale)
+            assert_parity(got, oracle.attention(q, k, v, c.scale, kv_valid_len=c.kv_valid_len),
+                          c.name)
+        else:
+            _sampled(oracle, c, per_head=4, full_heads=((1, 31),), tail_block=128)
 
 
 def test_longclip_sampled(oracle):
