@@ -34,6 +34,10 @@ static_assert(128 * kPPRegsProducer + 256 * kPPRegsSoftmax <= kPPThreads * kPPRe
               "register split exceeds the launch allocation");
 // every kPPExp2FmaEvery-th pair of exponentials runs on the FMA pipe (0 = none)
 constexpr int kPPExp2FmaEvery = 0;
+// P of each tile is published to the MMA warp in this many key parts (2 or 4), so that
+// the PV of the first parts overlaps the exponentials of the later ones
+constexpr int kPPParts = 2;
+static_assert(kPPParts == 2 || kPPParts == 4, "P parts");
 
 template <int D>
 struct PPSmem {
@@ -51,8 +55,8 @@ struct PPSmem {
   static constexpr int bVF = bKE + kStages;
   static constexpr int bVE = bVF + kStages;
   static constexpr int bSF = bVE + kStages;  // 2
-  static constexpr int bPF = bSF + 2;        // 4: [half * 2 + g]
-  static constexpr int bOF = bPF + 4;        // 2
+  static constexpr int bPF = bSF + 2;        // 2 * kPPParts: [part * 2 + g]
+  static constexpr int bOF = bPF + 2 * kPPParts;  // 2
   static constexpr int bDrain = bOF + 2;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
@@ -102,8 +106,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(L::bQF + g), 1);
       mbar_init(bar(L::bSF + g), 1);
-      mbar_init(bar(L::bPF + g), kBlockM);      // P keys 0-63 of tile g
-      mbar_init(bar(L::bPF + 2 + g), kBlockM);  // P keys 64-127 of tile g
+      for (int part = 0; part < kPPParts; ++part)  // P keys of one part of tile g
+        mbar_init(bar(L::bPF + part * 2 + g), kBlockM);
       mbar_init(bar(L::bOF + g), 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
@@ -208,12 +212,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       };
       // waits for P_g (both halves) and issues its PV; false on a failed wait
       auto pv = [&](int g, int st, bool acc, uint32_t pph) -> bool {
-        if (!wt(bar(L::bPF + g), pph)) return false;
-        tc_fence_after();
-        pv_part(g, st, acc, 0, kBlockN / 32);
-        if (!wt(bar(L::bPF + 2 + g), pph)) return false;
-        tc_fence_after();
-        pv_part(g, st, acc, kBlockN / 32, kBlockN / 16);
+#pragma unroll
+        for (int part = 0; part < kPPParts; ++part) {
+          if (!wt(bar(L::bPF + part * 2 + g), pph)) return false;
+          tc_fence_after();
+          pv_part(g, st, acc, part * (kBlockN / 16 / kPPParts),
+                  (part + 1) * (kBlockN / 16 / kPPParts));
+        }
         return true;
       };
       bool ok = wt(bar(L::bKF + 0), 0) && wt(bar(L::bQF + 0), 0);
@@ -312,19 +317,22 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       const float2 nm2 = make_float2(-m_run, -m_run);
       const float2 sc2 = make_float2(sl2, sl2);
       // exponentials on the MUFU (argument and row sum in packed fp32 pairs); P is
-      // published to the MMA warp in two 64-key halves so the PV of the first half
-      // overlaps the exponentials of the second
+      // published to the MMA warp in kPPParts key parts so the PV of the first parts
+      // overlaps the exponentials of the later ones
       float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int c = 0; c < kBlockN / 64; ++c) {
-        uint32_t pk0[16], pk1[16];
-        exp2_pack16<kPPExp2FmaEvery>(&s[c * 64], sc2, nm2, la, lb, pk0);
-        exp2_pack16<kPPExp2FmaEvery>(&s[c * 64 + 32], sc2, nm2, la, lb, pk1);
-        tmem_st16(trow + colS + c * 32, pk0);
-        tmem_st16(trow + colS + c * 32 + 16, pk1);
+      for (int part = 0; part < kPPParts; ++part) {
+        constexpr int kChunks = kBlockN / 32 / kPPParts;  // 32-key chunks per part
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int ch = part * kChunks + c;
+          uint32_t pk[16];
+          exp2_pack16<kPPExp2FmaEvery>(&s[ch * 32], sc2, nm2, la, lb, pk);
+          tmem_st16(trow + colS + ch * 16, pk);
+        }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::bPF + c * 2 + g));
+        mbar_arrive(bar(L::bPF + part * 2 + g));
       }
       l_run += (la.x + la.y) + (lb.x + lb.y);
     }
