@@ -34,7 +34,6 @@ namespace ltx {
 
 constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per tile
-constexpr int kFwdThreads = 192;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
 constexpr int kMinSmemFor1Cta = 120 * 1024;  // forces one CTA per SM (TMEM holds 512 columns)
 
@@ -56,27 +55,36 @@ struct FwdParams {
 };
 
 // kSBuf = 2: S double buffered (QK of tile j+1 overlaps the softmax of tile j), 512
-// TMEM columns, one CTA per SM.  kSBuf = 1: one S buffer, 256 TMEM columns and two K/V
-// stages, so that two CTAs share an SM and interleave their QK -> softmax -> PV chains
-// (head_dim 64 only: shared memory and registers must fit twice).
+// TMEM columns, one CTA per SM, 192 threads (producer, MMA, four softmax warps).
+// kSBuf = 1: one S buffer, 256 TMEM columns, 256 threads (producer, MMA and two idle
+// warps in the first warpgroup, which hands registers to the softmax warpgroup), three K
+// and two V stages, so that two CTAs share an SM and interleave their
+// QK -> softmax -> PV chains (head_dim 64 only: shared memory and registers fit twice).
 template <int D, int kSBuf = 2>
 struct FwdSmem {
   static_assert(kSBuf == 2 || (kSBuf == 1 && D == 64), "S buffers");
+  static constexpr int kThreads = kSBuf == 1 ? 256 : 192;
+  static constexpr int kSoftmaxWarp0 = kSBuf == 1 ? 4 : 2;  // first softmax warp
+  // kSBuf == 1: 2 CTAs x 256 threads x 128 registers at launch; setmaxnreg moves the first
+  // warpgroup to 56 and the softmax warpgroup to 200 (56 + 200 = 2 x 128)
   static constexpr int kBoxes = D / 64;             // 128-byte (64 x bf16) column boxes per row
   static constexpr int kBoxBytes = kBlockM * 128;   // one 128-row x 64-column box
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kStages = kSBuf == 1 ? 2 : (D == 64) ? 3 : 2;
+  static constexpr int kKStages = kSBuf == 1 ? 3 : (D == 64) ? 3 : 2;
+  static constexpr int kVStages = kSBuf == 1 ? 2 : (D == 64) ? 3 : 2;
+  // the producer issues K this many tiles ahead of V (K is needed a softmax earlier)
+  static constexpr int kKAhead = kKStages - kVStages;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
+  static constexpr int kV = kK + kKStages * kTileBytes;
+  static constexpr int kBar = kV + kVStages * kTileBytes;
   // barriers
   static constexpr int bQ = 0;
   static constexpr int bKF = 1;
-  static constexpr int bKE = bKF + kStages;
-  static constexpr int bVF = bKE + kStages;
-  static constexpr int bVE = bVF + kStages;
-  static constexpr int bSF = bVE + kStages;  // kSBuf
+  static constexpr int bKE = bKF + kKStages;
+  static constexpr int bVF = bKE + kKStages;
+  static constexpr int bVE = bVF + kVStages;
+  static constexpr int bSF = bVE + kVStages;  // kSBuf
   static constexpr int bPF = bSF + 2;        // kSBuf
   static constexpr int bOD = bPF + 2;        // O updated by a PV
   static constexpr int bOF = bOD + 1;        // final PV done
@@ -187,7 +195,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
 }
 
 template <int D, bool kSplit, int kSBuf = 2>
-__global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
+__global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
     fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams p) {
@@ -212,9 +220,11 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::bQ), 1);
-    for (int s = 0; s < L::kStages; ++s) {
+    for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::bKF + s), 1);
       mbar_init(bar(L::bKE + s), 1);
+    }
+    for (int s = 0; s < L::kVStages; ++s) {
       mbar_init(bar(L::bVF + s), 1);
       mbar_init(bar(L::bVE + s), 1);
     }
@@ -241,6 +251,7 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    if constexpr (kSBuf == 1) setmaxnreg_dec<56>();
     if (lane == 0 && !*abort_flag) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -249,41 +260,48 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
       for (int bx = 0; bx < L::kBoxes; ++bx)
         tma_load_4d(sbase + L::kQ + bx * L::kBoxBytes, &tm_q, bar(L::bQ), bx * 64, h,
                     qt * kBlockM, b);
-      int last_k[L::kStages], last_v[L::kStages];
-      for (int s = 0; s < L::kStages; ++s) last_k[s] = last_v[s] = -1;
+      int last_k[L::kKStages], last_v[L::kVStages];
+      for (int s = 0; s < L::kKStages; ++s) last_k[s] = -1;
+      for (int s = 0; s < L::kVStages; ++s) last_v[s] = -1;
       bool ok = true;
+      int nk = 0;  // next K tile to load (K runs kKAhead tiles ahead of V)
       for (int j = 0; j < n && ok; ++j) {
-        const int st = j % L::kStages;
-        const uint32_t ph = (uint32_t)(j / L::kStages) & 1u;
-        const int kv0 = (kv_begin + j) * kBlockN;
-        ok = mbar_wait(bar(L::bKE + st), ph ^ 1u, ctl);
+        for (; ok && nk < n && nk <= j + L::kKAhead; ++nk) {
+          const int st = nk % L::kKStages;
+          ok = mbar_wait(bar(L::bKE + st), ((uint32_t)(nk / L::kKStages) & 1u) ^ 1u, ctl);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar(L::bKF + st), L::kTileBytes);
+          for (int bx = 0; bx < L::kBoxes; ++bx)
+            tma_load_4d(sbase + L::kK + st * L::kTileBytes + bx * L::kBoxBytes, &tm_k,
+                        bar(L::bKF + st), bx * 64, h, (kv_begin + nk) * kBlockN, b);
+          last_k[st] = nk;
+        }
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::bKF + st), L::kTileBytes);
-        for (int bx = 0; bx < L::kBoxes; ++bx)
-          tma_load_4d(sbase + L::kK + st * L::kTileBytes + bx * L::kBoxBytes, &tm_k,
-                      bar(L::bKF + st), bx * 64, h, kv0, b);
-        last_k[st] = j;
-        ok = mbar_wait(bar(L::bVE + st), ph ^ 1u, ctl);
+        const int sv = j % L::kVStages;
+        ok = mbar_wait(bar(L::bVE + sv), ((uint32_t)(j / L::kVStages) & 1u) ^ 1u, ctl);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::bVF + st), L::kTileBytes);
+        mbar_arrive_expect_tx(bar(L::bVF + sv), L::kTileBytes);
         for (int bx = 0; bx < L::kBoxes; ++bx)
-          tma_load_4d(sbase + L::kV + st * L::kTileBytes + bx * L::kBoxBytes, &tm_v,
-                      bar(L::bVF + st), bx * 64, h, kv0, b);
-        last_v[st] = j;
+          tma_load_4d(sbase + L::kV + sv * L::kTileBytes + bx * L::kBoxBytes, &tm_v,
+                      bar(L::bVF + sv), bx * 64, h, (kv_begin + j) * kBlockN, b);
+        last_v[sv] = j;
       }
       if (!ok) {
         // let every copy this thread started land before shared memory is released
-        for (int s = 0; s < L::kStages; ++s) {
+        for (int s = 0; s < L::kKStages; ++s)
           if (last_k[s] >= 0)
-            mbar_wait_drain(bar(L::bKF + s), (uint32_t)(last_k[s] / L::kStages) & 1u, p.timeout_ns);
+            mbar_wait_drain(bar(L::bKF + s), (uint32_t)(last_k[s] / L::kKStages) & 1u,
+                            p.timeout_ns);
+        for (int s = 0; s < L::kVStages; ++s)
           if (last_v[s] >= 0)
-            mbar_wait_drain(bar(L::bVF + s), (uint32_t)(last_v[s] / L::kStages) & 1u, p.timeout_ns);
-        }
+            mbar_wait_drain(bar(L::bVF + s), (uint32_t)(last_v[s] / L::kVStages) & 1u,
+                            p.timeout_ns);
         mbar_wait_drain(bar(L::bQ), 0, p.timeout_ns);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    if constexpr (kSBuf == 1) setmaxnreg_dec<56>();
     if (lane == 0 && !*abort_flag) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
@@ -296,8 +314,8 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
       auto pv = [&](int t) -> bool {
         const int sb = t % kSBuf;
         if (!mbar_wait(bar(L::bPF + sb), (uint32_t)(t / kSBuf) & 1u, ctl)) return false;
-        const int st = t % L::kStages;
-        if (!mbar_wait(bar(L::bVF + st), (uint32_t)(t / L::kStages) & 1u, ctl)) return false;
+        const int st = t % L::kVStages;
+        if (!mbar_wait(bar(L::bVF + st), (uint32_t)(t / L::kVStages) & 1u, ctl)) return false;
         tc_fence_after();
         const uint32_t v_off = (uint32_t)st * L::kTileBytes;
 #pragma unroll
@@ -316,8 +334,8 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
           ok = pv(j - 1);
           if (!ok) break;
         }
-        const int st = j % L::kStages;
-        ok = mbar_wait(bar(L::bKF + st), (uint32_t)(j / L::kStages) & 1u, ctl);
+        const int st = j % L::kKStages;
+        ok = mbar_wait(bar(L::bKF + st), (uint32_t)(j / L::kKStages) & 1u, ctl);
         if (!ok) break;
         tc_fence_after();
         const int sb = j % kSBuf;
@@ -341,8 +359,11 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
         mbar_wait_drain(bar(L::bDrain), 0, p.timeout_ns);
       }
     }
+  } else if (kSBuf == 1 && warp < L::kSoftmaxWarp0) {
+    setmaxnreg_dec<56>();  // warps 2-3: idle members of the first warpgroup
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    if constexpr (kSBuf == 1) setmaxnreg_inc<200>();
     const int wq = warp & 3;  // TMEM lane quadrant this warp may access
     const int row = wq * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
@@ -357,33 +378,18 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
       tc_fence_after();
       const uint32_t tS = trow + sb * 128;
       const int lim = p.kv_valid - (kv_begin + j) * kBlockN;  // valid keys in this tile
-      // kSBuf == 2: the whole 128-score row stays in registers.  kSBuf == 1 (two CTAs
-      // per SM, fewer registers): 64-column halves, read twice from TMEM.
-      float s[kSBuf == 2 ? kBlockN : 64];
-      float mx;
-      if constexpr (kSBuf == 2) {
+      // the whole 128-score row stays in registers
+      float s[kBlockN];
 #pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c)
-          tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-        tmem_ld_wait();
-        if (lim < kBlockN) {
+      for (int c = 0; c < kBlockN / 32; ++c)
+        tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+      tmem_ld_wait();
+      if (lim < kBlockN) {
 #pragma unroll
-          for (int c = 0; c < kBlockN; ++c)
-            if (c >= lim) s[c] = -INFINITY;
-        }
-        mx = row_max<kBlockN>(s) * sl2;
-      } else {
-        float m = -INFINITY;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          tmem_ld32(tS + hf * 64, *reinterpret_cast<float(*)[32]>(&s[0]));
-          tmem_ld32(tS + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
-          tmem_ld_wait();
-          if (lim < (hf + 1) * 64) mask_keys<2>(s, lim - hf * 64);
-          m = fmaxf(m, row_max<64>(s));
-        }
-        mx = m * sl2;
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= lim) s[c] = -INFINITY;
       }
+      float mx = row_max<kBlockN>(s) * sl2;
       if (j == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, mx > m_run + kRescaleThreshold)) {
@@ -412,28 +418,11 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
       const float2 nm2 = make_float2(-m_run, -m_run);
       const float2 sc2 = make_float2(sl2, sl2);
       float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
-      if constexpr (kSBuf == 2) {
 #pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c) {
-          uint32_t pk[16];
-          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
-          tmem_st16(tS + c * 16, pk);
-        }
-      } else {
-        // P of half hf lands on columns [32 hf, 32 hf + 32), read in the first half
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          tmem_ld32(tS + hf * 64, *reinterpret_cast<float(*)[32]>(&s[0]));
-          tmem_ld32(tS + hf * 64 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
-          tmem_ld_wait();
-          if (lim < (hf + 1) * 64) mask_keys<2>(s, lim - hf * 64);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t pk[16];
-            exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
-            tmem_st16(tS + hf * 32 + c * 16, pk);
-          }
-        }
+      for (int c = 0; c < kBlockN / 32; ++c) {
+        uint32_t pk[16];
+        exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+        tmem_st16(tS + c * 16, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -470,7 +459,7 @@ __global__ void __launch_bounds__(kFwdThreads, 3 - kSBuf)
         }
         fence_proxy_async_smem();
         named_bar_sync(1, kBlockM);
-        if (threadIdx.x == 64) {
+        if (threadIdx.x == L::kSoftmaxWarp0 * 32) {
           for (int bx = 0; bx < L::kBoxes; ++bx)
             tma_store_4d(&tm_o, sbase + L::kQ + bx * L::kBoxBytes, bx * 64, h, qt * kBlockM, b);
           tma_store_commit();

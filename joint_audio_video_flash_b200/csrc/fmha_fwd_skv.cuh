@@ -110,15 +110,6 @@ struct SkvCursor {
   }
 };
 
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
-}
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
-}
-
 template <int D, int NKV>
 __global__ void __launch_bounds__(kSkvThreads, 1)
     fmha_fwd_skv_sm100(const __grid_constant__ CUtensorMap tm_q,

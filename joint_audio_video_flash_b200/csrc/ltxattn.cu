@@ -142,7 +142,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
   dim3 grid(p.n_q_tiles, p.heads, p.batch * p.num_splits);
   ltx::fmha_fwd_sm100<D, kSplit, kSBuf>
-      <<<grid, ltx::kFwdThreads, FwdSmem<D, kSBuf>::kAlloc, stream>>>(tq, tk, tv, to, p);
+      <<<grid, FwdSmem<D, kSBuf>::kThreads, FwdSmem<D, kSBuf>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 

@@ -193,6 +193,17 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
+// Register reallocation between warpgroups (every warp of a warpgroup executes the same
+// one); the increases must fit in what the decreases and the launch allocation free.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // tcgen05: TMEM allocation
 // ----------------------------------------------------------------------------
