@@ -106,7 +106,7 @@ bool encode_bshd(const Context& c, CUtensorMap* map, const void* base, int len, 
 // over-splitting.  Cost model: waves x (tiles per part + fixed per-CTA overhead).
 int plan_splits(int units, int n_kv_tiles, int num_sms) {
   if (n_kv_tiles < 4 || units >= num_sms) return 1;
-  const int kOverheadTiles = 2;
+  const int kOverheadTiles = 4;  // pipeline fill + partial write-out, in key tiles (measured)
   int best = 1;
   long long best_cost = -1;
   for (int s = 1; s <= std::min(n_kv_tiles, 64); ++s) {
@@ -340,11 +340,13 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   p.status = c->d_status;
   p.timeout_ns = kDefaultTimeoutNs;
 
-  const int units = p.n_q_tiles * heads * batch;
   // head_dim 64 with a long key side and a short query side (v2a): one S buffer per
   // CTA and two CTAs per SM, so the split planner counts two CTA slots per SM
   const bool dual = head_dim == 64 && p.n_kv_tiles > ltx::kSkvMaxKvTiles &&
                     p.n_q_tiles <= kDualMaxQTiles;
+  // CTAs per key-range part: the two-query-tile kernel takes query tiles in pairs
+  const int q_ctas = (!dual && p.n_q_tiles >= 2) ? (p.n_q_tiles + 1) / 2 : p.n_q_tiles;
+  const int units = q_ctas * heads * batch;
   int splits = num_splits > 0 ? std::min(num_splits, p.n_kv_tiles)
                               : plan_splits(units, p.n_kv_tiles, (dual ? 2 : 1) * c->num_sms);
   p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
