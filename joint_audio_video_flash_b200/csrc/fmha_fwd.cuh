@@ -136,43 +136,14 @@ __device__ __forceinline__ float row_max(const float* s) {
   return fmax3(fmaxf(m[0], m[1]), m[2], m[3]);
 }
 
-// 2^x for a pair of fp32 values on the FMA pipe instead of the MUFU (which the
-// exponentials of attention keep saturated on sm_100).  Range reduction x = n + f with
-// n = round(x), obtained by adding and subtracting the shifter 1.5 * 2^23 (the FADD
-// rounds to nearest), f in [-1/2, 1/2]; 2^f from the cubic 1 + c1 f + c2 f^2 + c3 f^3
-// whose coefficients are the minimax fit of the relative error on [-1/2, 1/2] with the
-// constant term held at 1 (linear programming on a dense grid; max relative error
-// 1.01e-4 in fp32 Horner form, a twentieth of a bf16 ulp); 2^n applied by adding n << 23
-// to the bit pattern (the shifted sum's low mantissa bits hold n).  x is clamped at
-// -127, where f = 0 and p = 1 give the bit pattern of +0, so a masked key (-inf)
-// yields exactly 0.  Valid for x <= 127.
-__device__ __forceinline__ float2 exp2_fma_pair(float2 x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float kC1 = 0.6932829f, kC2 = 0.24221097f, kC3 = 0.05500906f;
-  x = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
-  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
-  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);  // x - n, exact
-  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // 32 scores -> p = 2^(s*scale_log2 - m) as 16 packed bf16 pairs; the fp32 p are added
 // to the two packed row-sum accumulators.  Argument and sums use packed fp32 pairs.
-// kFmaEvery > 0 moves every kFmaEvery-th pair's exponentials from the MUFU to the FMA
-// pipe (exp2_fma_pair).
-template <int kFmaEvery = 0>
 __device__ __forceinline__ void exp2_pack16(const float* s, float2 sc2, float2 nm2, float2& la,
                                             float2& lb, uint32_t (&pk)[16]) {
 #pragma unroll
   for (int x = 0; x < 16; ++x) {
     const float2 a = __ffma2_rn(make_float2(s[2 * x], s[2 * x + 1]), sc2, nm2);
-    const float2 e = (kFmaEvery > 0 && x % (kFmaEvery > 0 ? kFmaEvery : 1) == kFmaEvery - 1)
-                         ? exp2_fma_pair(a)
-                         : make_float2(ex2(a.x), ex2(a.y));
+    const float2 e = make_float2(ex2(a.x), ex2(a.y));
     if (x & 1)
       lb = __fadd2_rn(lb, e);
     else

@@ -32,8 +32,6 @@ constexpr int kPPRegsProducer = 88;  // warps 0-3 after setmaxnreg.dec
 constexpr int kPPRegsSoftmax = 208;  // warps 4-11 after setmaxnreg.inc
 static_assert(128 * kPPRegsProducer + 256 * kPPRegsSoftmax <= kPPThreads * kPPRegsLaunch,
               "register split exceeds the launch allocation");
-// every kPPExp2FmaEvery-th pair of exponentials runs on the FMA pipe (0 = none)
-constexpr int kPPExp2FmaEvery = 0;
 // P of each tile is published to the MMA warp in this many key parts (2 or 4), so that
 // the PV of the first parts overlaps the exponentials of the later ones
 constexpr int kPPParts = 2;
@@ -327,7 +325,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int c = 0; c < kChunks; ++c) {
           const int ch = part * kChunks + c;
           uint32_t pk[16];
-          exp2_pack16<kPPExp2FmaEvery>(&s[ch * 32], sc2, nm2, la, lb, pk);
+          exp2_pack16(&s[ch * 32], sc2, nm2, la, lb, pk);
           tmem_st16(trow + colS + ch * 16, pk);
         }
         tmem_st_wait();

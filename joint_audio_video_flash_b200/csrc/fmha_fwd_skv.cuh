@@ -37,9 +37,6 @@ constexpr int kSkvRegsLaunch = 128;  // 65536 / 512
 constexpr int kSkvRegsIssue = 56;    // warps 0-3
 constexpr int kSkvRegsEpi = 104;     // warps 12-15
 constexpr int kSkvRegsSoftmax = 176; // warps 4-11
-// every kSkvExp2FmaEvery-th pair of exponentials of the two-key-tile path runs on the FMA
-// pipe (0 = none)
-constexpr int kSkvExp2FmaEvery = 0;
 static_assert(128 * kSkvRegsIssue + 128 * kSkvRegsEpi + 256 * kSkvRegsSoftmax <=
                   kSkvThreads * kSkvRegsLaunch,
               "register split exceeds the launch allocation");
@@ -347,7 +344,7 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
           uint32_t pk[16];
-          exp2_pack16<kSkvExp2FmaEvery>(&s[c * 32], sc2, nm2, la, lb, pk);
+          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
           tmem_st16(trow + c * 16, pk);
         }
 #pragma unroll
@@ -383,7 +380,7 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
           uint32_t pk[16];
-          exp2_pack16<kSkvExp2FmaEvery>(&s[c * 32], sc2, nm2, la, lb, pk);
+          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
           tmem_st16(trow + 64 + c * 16, pk);
         }
       }
