@@ -36,7 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, keyed by
 # the hash of the kernel sources it was taken on; reported as null once the sources change.
 TRAFFIC = {
-    "video_self": {"src": "c5524e8f43c297c3", "bytes_per_token": (201.557504e6 + 48.422400e6) / 8192,
+    "video_self": {"src": "3fe5540a7028fb95", "bytes_per_token": (201.515264e6 + 46.888448e6) / 8192,
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
 }
 KERNEL_SOURCES = ("joint_audio_video_flash_b200/csrc/fmha_fwd_pp.cuh",
