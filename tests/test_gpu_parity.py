@@ -144,6 +144,19 @@ def test_forced_key_splits(oracle, splits):
     assert_parity(got, ref, f"splits={splits}")
 
 
+def test_split_parts_across_alternating_shapes(oracle):
+    # one query tile over a long key side, split into key-range parts; calls of alternating
+    # shapes reuse the per-stream workspace of partials
+    shapes = [(2, 4, 126, 2048, 2000, 3), (3, 5, 100, 3000, 2999, 4), (2, 4, 126, 2048, 2000, 5),
+              (1, 2, 64, 640, 600, 5)]
+    for b, h, lq, lkv, valid, splits in shapes + shapes[:1]:
+        q, k, v = synth.make_qkv(b, lq, lkv, h, 64, seed=lq + lkv + h, kv_valid=valid)
+        got, used = gpu_run(q, k, v, valid, 0.125, num_splits=splits)
+        assert used > 1
+        assert_parity(got, oracle.attention(q, k, v, 0.125, kv_valid_len=valid),
+                      f"b{b} h{h} q{lq} kv{lkv} splits {used}")
+
+
 @pytest.mark.parametrize("d,splits", [(64, 3), (128, 2), (128, 7)])
 def test_forced_key_splits_two_query_tiles(oracle, d, splits):
     # query side of several tiles (odd count: the last CTA's second tile is empty)
