@@ -1,0 +1,63 @@
+"""The JSON line bench.py prints: every key its consumers read, with sane values.
+
+The reference arm (the fp64 oracle on a bounded sample) runs on CPU; the GPU arm is run on
+the tiny workload (marked gpu).
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+COMMON = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+          "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "e2e"}
+
+
+def _run(args, timeout):
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(k, None)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                         env=env, capture_output=True, text=True, timeout=timeout)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    d = _run(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "0",
+              "--reference-budget-s", "4"], timeout=600)
+    assert COMMON <= set(d)
+    assert d["impl"] == "reference"
+    assert d["warmup"] >= 3 and d["steps"] == 2
+    assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.gpu
+def test_gpu_arm_line():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    d = _run(["--workload", "tiny", "--steps", "3", "--warmup", "3", "--cpu-seconds", "2"],
+             timeout=900)
+    assert COMMON <= set(d) and "impl" not in d
+    assert d["n_gpus"] == 1 and d["scaling"] == "weak" and d["dtype"] == "bf16"
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    r = d["roofline"]
+    assert r["bound"] in ("tensor", "hbm") and r["achieved"] > 0 and r["peak"] > 0
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    e = d["e2e"]
+    assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    # four calls per step, one launch each (no key-range parts at these sizes)
+    assert d["gpu_launches"] == 4 * d["steps"]
+    assert set(d["per_call"]) == {"video_self", "audio_self", "v2a", "a2v"}
+    assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
