@@ -281,6 +281,41 @@ def test_longclip_sampled(oracle):
                  tail_block=144 if c.q_len > 256 else 0)
 
 
+def test_concurrent_streams_use_separate_workspaces(oracle):
+    # key-range splits on two streams at once: each stream has its own partials workspace
+    cases = [synth.make_qkv(2, 126, 4096, 4, 64, seed=51, kv_valid=4000),
+             synth.make_qkv(1, 300, 3000, 3, 128, seed=52, kv_valid=2990)]
+    valids, scales = [4000, 2990], [0.125, 1.0 / np.sqrt(128)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    dev = [[t.cuda() for t in c] for c in cases]
+    outs = [torch.empty_like(d[0]) for d in dev]
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for i in range(2):
+            with torch.cuda.stream(streams[i]):
+                ltxattn.forward(*dev[i], outs[i], kv_valid_len=valids[i], scale=scales[i],
+                                num_splits=4 + rep, stream=streams[i])
+    torch.cuda.synchronize()
+    ltxattn.check()
+    for i in range(2):
+        q, k, v = cases[i]
+        assert_parity(outs[i].cpu(), oracle.attention(q, k, v, scales[i], kv_valid_len=valids[i]),
+                      f"stream {i}")
+
+
+def test_context_survives_destroy_and_create(oracle):
+    q, k, v = synth.make_qkv(1, 200, 1000, 2, 64, seed=53)
+    ref = oracle.attention(q, k, v, 0.125)
+    for _ in range(2):
+        ltxattn.destroy()
+        with pytest.raises(ltxattn.LtxAttnError) as e:
+            ltxattn.forward(q.cuda(), k.cuda(), v.cuda(), scale=0.125)
+        assert e.value.status == ltxattn.ERR_NOT_INITIALIZED
+        ltxattn.create()
+        got, _ = gpu_run(q, k, v, 1000, 0.125, num_splits=3)
+        assert_parity(got, ref, "after re-create")
+
+
 def test_errors_on_device():
     q = torch.zeros(1, 64, 2, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ltxattn.LtxAttnError) as e:
