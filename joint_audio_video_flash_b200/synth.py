@@ -55,3 +55,32 @@ def sample_rows(batch: int, q_len: int, heads: int, per_head: int, seed: int,
             i = torch.randperm(q_len, generator=g)[:n].to(torch.int64)
             idx.append((b * q_len + i) * heads + h)
     return torch.unique(torch.cat(idx))
+
+
+def rope_tables(length: int, head_dim: int, base: float = 10000.0):
+    """Rotary tables for positions 0..length-1: cos, sin of p * base^(-2i/head_dim), fp32.
+
+    Shape [length, head_dim // 2]; pair i of every head at position p turns by that angle.
+    These are inputs to the rotary step (the caller owns the positional scheme), computed in
+    fp64 and rounded to fp32.
+    """
+    half = head_dim // 2
+    inv_freq = base ** (-torch.arange(half, dtype=torch.float64) * 2.0 / head_dim)
+    ang = torch.arange(length, dtype=torch.float64)[:, None] * inv_freq[None, :]
+    return torch.cos(ang).to(torch.float32), torch.sin(ang).to(torch.float32)
+
+
+def make_qk_prologue_inputs(batch: int, seq_len: int, heads: int, head_dim: int, seed: int):
+    """(q, k, q_weight, k_weight, cos, sin) for the QK-norm + rotary prologue.
+
+    q, k: bf16 N(0, 1) [batch, seq_len, heads, head_dim]; weights: bf16 1 + 0.1 N(0, 1) over
+    heads * head_dim; cos, sin: :func:`rope_tables` for positions 0..seq_len-1.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = bf16_normal((batch, seq_len, heads, head_dim), g)
+    k = bf16_normal((batch, seq_len, heads, head_dim), g)
+    wq = (1.0 + 0.1 * torch.randn(heads * head_dim, generator=g)).to(torch.bfloat16)
+    wk = (1.0 + 0.1 * torch.randn(heads * head_dim, generator=g)).to(torch.bfloat16)
+    cos, sin = rope_tables(seq_len, head_dim)
+    return q, k, wq, wk, cos, sin
