@@ -7,6 +7,7 @@ run back to back on one stream through the C ABI (libltxattn.so).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...     # the fp64 CPU oracle, timed on a sample
+    python bench.py --workload qk_prologue   # the QK-norm + rotary prologue alone (GB/s)
 
 Prints one JSON line (rank 0).  ``value`` is the whole-job TFLOP/s (algorithmic
 FLOPs of all ranks / max-over-ranks device time); the timed region holds exactly
@@ -484,6 +485,105 @@ def run_ltxattn(args):
         dist.destroy_process_group()
 
 
+def run_prologue(args):
+    """The QK-norm + rotary prologue at the video stream's size (HBM-bound streaming kernel)."""
+    import torch
+
+    from joint_audio_video_flash_b200 import build, ltxattn, synth
+    world, rank, local = dist_setup(args.gpus)
+    build.build()
+    b, l, h, d = 2, 15360, 32, 128
+    q, k, wq, wk, cos, sin = synth.make_qk_prologue_inputs(b, l, h, d, seed=21)
+    dev = torch.device("cuda", local)
+    dq, dk, dwq, dwk, dcos, dsin = (t.to(dev) for t in (q, k, wq, wk, cos, sin))
+    qo, ko = torch.empty_like(dq), torch.empty_like(dk)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ltxattn.qk_norm_rope(dq, dk, dwq, dwk, dcos, dsin, qo, ko)
+
+    if args.once:  # one launch, no timing: the command the Nsight Compute captures run
+        step()
+        torch.cuda.synchronize()
+        print(json.dumps({"workload": args.workload, "once": True}))
+        return
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(None) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    # algorithmic bytes: q and k read and written once (bf16); weights and tables are 0.1 %
+    step_bytes = 4.0 * dq.numel() * 2 + 2 * dwq.numel() * 2 + 2 * dcos.numel() * 4
+    value = step_bytes * args.steps * world / (total_ms * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    # end to end: inputs uploaded from pinned memory, outputs downloaded, every step
+    hq, hk = q.pin_memory(), k.pin_memory()
+    oq, ok_ = torch.empty(q.shape, dtype=q.dtype, pin_memory=True), \
+        torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        step()
+        oq.copy_(qo, non_blocking=True)
+        ok_.copy_(ko, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    line = {
+        "metric": "qk norm + rotary prologue GB/s", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "qk_prologue",
+                   "description": "queries and keys of the video stream, B2 x 15360 tokens x "
+                                  "32 heads x 128: RMSNorm over heads*dim, rotary on channel "
+                                  "pairs (a reading; see the header)",
+                   "l2": "inputs larger than L2 (q and k are 252 MB each)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": value, "peak": hbm, "unit": "GB/s",
+                     "frac": value / hbm, "traffic": None, "kernel": "qk_norm_rope<16>",
+                     "algorithmic_bytes": step_bytes, "peak_source": f"{peak_src} hbm_gbs"},
+        "e2e": {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * q.numel() * 2, "d2h_bytes_per_step": 2 * q.numel() * 2},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import qk_prologue as qp
+        blk, done, secs = 512, 0, 0.0
+        while done < l and secs < args.cpu_seconds:
+            sl = slice(done, min(l, done + blk))
+            t_start = time.perf_counter()
+            qp.rms_norm_rope(q[:, sl], wq, cos[sl], sin[sl], 1e-6)
+            qp.rms_norm_rope(k[:, sl], wk, cos[sl], sin[sl], 1e-6)
+            secs += time.perf_counter() - t_start
+            done = sl.stop
+        line["cpu_baseline"] = {"value": step_bytes * (done / l) / secs / 1e9, "unit": "GB/s",
+                                "cores": 1, "kind": "oracle",
+                                "sample": f"token positions 0..{done - 1} of {l} in blocks of "
+                                          f"{blk}, both batch elements, q and k; numpy fp64, "
+                                          f"{secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -498,7 +598,9 @@ def main():
                     help="run each call of the workload once and exit (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
-    if args.impl == "reference":
+    if args.workload == "qk_prologue" and args.impl != "reference":
+        run_prologue(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ltxattn(args)

@@ -144,6 +144,38 @@ LTXATTN_API const char* ltxattn_status_string(int status);
  */
 LTXATTN_API int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltxattn_stream_t stream);
 
+/*
+ * Norm and rotary step of the queries and keys ahead of attention, both tensors in one
+ * launch.  The LTX-2.5 DiT attends with "normed and rotated" queries and keys and keeps
+ * RoPE tables per latent grid ("feat(ltx2): tile-parallel video VAE and the two-stage
+ * pipeline", commit "Onboard Lightricks LTX-2.5"); the pages fix neither the norm nor the
+ * rotary layout, and this call computes the following reading.  For each tensor x (q or k),
+ * batch element b and token l, over the token's whole inner dimension heads * head_dim:
+ *     r = sqrt(mean_{h,d} x[b,l,h,d]^2 + eps),   y[h,d] = x[b,l,h,d] / r * weight[h*head_dim + d]
+ * then within every head, for each pair of adjacent channels (2i, 2i+1):
+ *     out[2i]   = y[2i] * cos[l,i] - y[2i+1] * sin[l,i]
+ *     out[2i+1] = y[2i] * sin[l,i] + y[2i+1] * cos[l,i]
+ * The tables carry the positional scheme (1-D or per-grid 3-D angles), so the caller owns it.
+ *
+ *   q, k          bf16 [batch, seq_len, heads, head_dim] (device), read
+ *   q_out, k_out  bf16, same shape (device), written; each may be its own input (in place),
+ *                 but must not otherwise overlap q, k or each other
+ *   q_weight, k_weight  bf16 [heads * head_dim] (device)
+ *   cos_table, sin_table  fp32 [seq_len, head_dim / 2] (device)
+ *   heads * head_dim  one of 512, 1024, 2048, 4096 (UNSUPPORTED otherwise); head_dim a
+ *                 multiple of 8
+ *   eps           finite, >= 0
+ * Arithmetic in fp32, output rounded to bf16 (nearest even).  Needs no ltxattn_create.
+ * Pointers must be 16-byte aligned (MISALIGNED).  Checks run on the host before any
+ * CUDA call (INVALID_ARG, UNSUPPORTED, MISALIGNED); LTXATTN_ERR_CUDA on a failed launch.
+ * Asynchronous on `stream`.
+ */
+LTXATTN_API int ltxattn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
+                                     const void* q_weight, const void* k_weight,
+                                     const float* cos_table, const float* sin_table, int batch,
+                                     int seq_len, int heads, int head_dim, float eps,
+                                     ltxattn_stream_t stream);
+
 /* Size of the library's built-in scratch array used by ltxattn_forward_split_noalloc. */
 #define LTXATTN_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per GPU */
 

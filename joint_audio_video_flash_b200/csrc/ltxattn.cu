@@ -17,6 +17,7 @@
 #include "fmha_fwd.cuh"
 #include "fmha_fwd_pp.cuh"
 #include "fmha_fwd_skv.cuh"
+#include "qk_prologue.cuh"
 
 namespace {
 
@@ -53,7 +54,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_create",        "ltxattn_forward",          "ltxattn_forward_ex",
     "ltxattn_check",         "ltxattn_destroy",          "ltxattn_status_string",
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
-    "ltxattn_forward_split_noalloc",
+    "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -470,6 +471,56 @@ int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltxattn_stream_
   wait_probe_kernel<<<1, 32, 0, stream>>>(c->d_status, timeout_ns);
   if (cudaGetLastError() != cudaSuccess) return LTXATTN_ERR_CUDA;
   return read_and_clear_status(c, stream);
+}
+
+int ltxattn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
+                         const void* q_weight, const void* k_weight, const float* cos_table,
+                         const float* sin_table, int batch, int seq_len, int heads, int head_dim,
+                         float eps, ltxattn_stream_t stream_) {
+  const void* ptrs[8] = {q, k, q_out, k_out, q_weight, k_weight, cos_table, sin_table};
+  for (const void* ptr : ptrs)
+    if (!ptr) return LTXATTN_ERR_INVALID_ARG;
+  if (batch < 1 || seq_len < 1 || heads < 1 || head_dim < 1) return LTXATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || eps < 0.0f) return LTXATTN_ERR_INVALID_ARG;
+  if (seq_len > LTXATTN_MAX_LEN || batch > LTXATTN_MAX_BATCH || heads > LTXATTN_MAX_HEADS)
+    return LTXATTN_ERR_UNSUPPORTED;
+  const long long inner = (long long)heads * head_dim;
+  if (head_dim % 8 != 0 || (inner != 512 && inner != 1024 && inner != 2048 && inner != 4096))
+    return LTXATTN_ERR_UNSUPPORTED;
+  uintptr_t mis = 0;
+  for (const void* ptr : ptrs) mis |= reinterpret_cast<uintptr_t>(ptr);
+  if (mis & 15u) return LTXATTN_ERR_MISALIGNED;
+  const size_t nbytes = (size_t)batch * seq_len * inner * 2;
+  // each output may be its own input; no other overlap
+  if ((q_out != q && overlaps(q_out, nbytes, q, nbytes)) || overlaps(q_out, nbytes, k, nbytes) ||
+      (k_out != k && overlaps(k_out, nbytes, k, nbytes)) || overlaps(k_out, nbytes, q, nbytes) ||
+      overlaps(q_out, nbytes, k_out, nbytes))
+    return LTXATTN_ERR_INVALID_ARG;
+
+  ltx::PrologueParams p{};
+  p.x[0] = static_cast<const __nv_bfloat16*>(q);
+  p.x[1] = static_cast<const __nv_bfloat16*>(k);
+  p.out[0] = static_cast<__nv_bfloat16*>(q_out);
+  p.out[1] = static_cast<__nv_bfloat16*>(k_out);
+  p.w[0] = static_cast<const __nv_bfloat16*>(q_weight);
+  p.w[1] = static_cast<const __nv_bfloat16*>(k_weight);
+  p.cos_t = cos_table;
+  p.sin_t = sin_table;
+  p.rows = (long long)batch * seq_len;
+  p.seq_len = seq_len;
+  p.head_dim = head_dim;
+  p.eps = eps;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const long long blocks = (2 * p.rows + ltx::kPrologueWarps - 1) / ltx::kPrologueWarps;
+  if (blocks > 0x7fffffffLL) return LTXATTN_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)blocks), block(ltx::kPrologueWarps * 32);
+  switch (inner) {
+    case 512: ltx::qk_norm_rope<2><<<grid, block, 0, stream>>>(p); break;
+    case 1024: ltx::qk_norm_rope<4><<<grid, block, 0, stream>>>(p); break;
+    case 2048: ltx::qk_norm_rope<8><<<grid, block, 0, stream>>>(p); break;
+    default: ltx::qk_norm_rope<16><<<grid, block, 0, stream>>>(p); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
 int ltxattn_num_entry_points(void) {

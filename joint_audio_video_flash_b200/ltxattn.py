@@ -49,6 +49,8 @@ def load() -> ctypes.CDLL:
             lib.ltxattn_status_string.restype = ctypes.c_char_p
             lib.ltxattn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp]
             lib.ltxattn_num_entry_points.argtypes = []
+            lib.ltxattn_qk_norm_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
+                                                 cf, vp]
             lib.ltxattn_entry_point_name.argtypes = [ci]
             lib.ltxattn_entry_point_name.restype = ctypes.c_char_p
             _lib = lib
@@ -156,3 +158,41 @@ def forward_split_noalloc(q, k, v, out, *, kv_valid_len: int | None = None,
                   int(q_len), int(kv_len), int(kv_valid_len), int(batch), int(heads),
                   int(head_dim), ctypes.c_float(scale), int(num_splits),
                   vp(_stream_handle(stream))))
+
+
+def qk_norm_rope(q, k, q_weight, k_weight, cos, sin, q_out=None, k_out=None, *,
+                 eps: float = 1e-6, stream=None):
+    """Norm and rotary step of queries and keys (``ltxattn_qk_norm_rope``); returns (q', k').
+
+    q, k: bf16 CUDA [B, L, H, D]; weights: bf16 [H * D]; cos, sin: fp32 [L, D / 2].  The
+    outputs may be the inputs (in place).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda \
+                or t.dim() != 4 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous bf16 CUDA [batch, len, heads, dim] tensor")
+    if k.shape != q.shape:
+        raise ValueError("q and k must have the same shape")
+    batch, seq_len, heads, head_dim = q.shape
+    for name, t, dt, shape in (("q_weight", q_weight, torch.bfloat16, (heads * head_dim,)),
+                               ("k_weight", k_weight, torch.bfloat16, (heads * head_dim,)),
+                               ("cos", cos, torch.float32, (seq_len, head_dim // 2)),
+                               ("sin", sin, torch.float32, (seq_len, head_dim // 2))):
+        if (not isinstance(t, torch.Tensor) or t.dtype != dt or not t.is_cuda
+                or tuple(t.shape) != shape or not t.is_contiguous()):
+            raise TypeError(f"{name} must be a contiguous {dt} CUDA tensor of shape {shape}")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    for name, t in (("q_out", q_out), ("k_out", k_out)):
+        if t.dtype != torch.bfloat16 or t.shape != q.shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q")
+    st = load().ltxattn_qk_norm_rope(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(q_out.data_ptr()), ctypes.c_void_p(k_out.data_ptr()),
+        ctypes.c_void_p(q_weight.data_ptr()), ctypes.c_void_p(k_weight.data_ptr()),
+        ctypes.c_void_p(cos.data_ptr()), ctypes.c_void_p(sin.data_ptr()), int(batch),
+        int(seq_len), int(heads), int(head_dim), ctypes.c_float(eps),
+        ctypes.c_void_p(_stream_handle(stream)))
+    _check(st, "ltxattn_qk_norm_rope")
+    return q_out, k_out
