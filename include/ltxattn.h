@@ -162,9 +162,10 @@ LTXATTN_API int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltx
  *                 but must not otherwise overlap q, k or each other
  *   q_weight, k_weight  bf16 [heads * head_dim] (device)
  *   cos_table, sin_table  fp32 [seq_len, head_dim / 2] (device)
- *   heads * head_dim  one of 512, 1024, 2048, 4096 (UNSUPPORTED otherwise); head_dim a
+ *   heads * head_dim  one of 512, 1024, 2048, 4096, 8192 (UNSUPPORTED otherwise); head_dim a
  *                 multiple of 8
  *   eps           finite, >= 0
+ *   batch * seq_len  below 2^30 (UNSUPPORTED otherwise)
  * Arithmetic in fp32, output rounded to bf16 (nearest even).  Needs no ltxattn_create.
  * Pointers must be 16-byte aligned (MISALIGNED).  Checks run on the host before any
  * CUDA call (INVALID_ARG, UNSUPPORTED, MISALIGNED); LTXATTN_ERR_CUDA on a failed launch.

@@ -279,6 +279,44 @@ int read_and_clear_status(Context* c, cudaStream_t stream) {
   return LTXATTN_OK;
 }
 
+// Persistent grid of the prologue: as many CTAs as fit on the device at once (looked up
+// once per device and kernel), fewer when there are fewer row groups.  MIN_CTAS caps the
+// registers: 3 CTAs an SM (80 registers) streamed faster at 1024 and 8192 channels, 2 CTAs
+// (128 registers) at 512, 2048 and 4096, on B200.
+template <int CHUNKS, int WPR, int MIN_CTAS>
+int launch_prologue(const ltx::PrologueParams& p, cudaStream_t stream) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static int resident[kMaxDevices];  // CTAs resident on the whole device; 0 = not looked up
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  int ctas = 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (resident[dev] == 0) {
+      int sms = 0, per_sm = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ltx::qk_norm_rope<CHUNKS, WPR, MIN_CTAS>,
+                                                        ltx::kPrologueWarps * 32, 0) !=
+              cudaSuccess ||
+          sms < 1 || per_sm < 1) {
+        cudaGetLastError();
+        return LTXATTN_ERR_CUDA;
+      }
+      resident[dev] = sms * per_sm;
+    }
+    ctas = resident[dev];
+  }
+  constexpr int kRowsPerCta = ltx::PrologueRow<CHUNKS, WPR>::kRowsPerCta;
+  const int groups = (2 * p.rows + kRowsPerCta - 1) / kRowsPerCta;
+  const unsigned grid = (unsigned)std::min(groups, ctas);
+  ltx::qk_norm_rope<CHUNKS, WPR, MIN_CTAS><<<grid, ltx::kPrologueWarps * 32, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -485,7 +523,8 @@ int ltxattn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
   if (seq_len > LTXATTN_MAX_LEN || batch > LTXATTN_MAX_BATCH || heads > LTXATTN_MAX_HEADS)
     return LTXATTN_ERR_UNSUPPORTED;
   const long long inner = (long long)heads * head_dim;
-  if (head_dim % 8 != 0 || (inner != 512 && inner != 1024 && inner != 2048 && inner != 4096))
+  if (head_dim % 8 != 0 ||
+      (inner != 512 && inner != 1024 && inner != 2048 && inner != 4096 && inner != 8192))
     return LTXATTN_ERR_UNSUPPORTED;
   uintptr_t mis = 0;
   for (const void* ptr : ptrs) mis |= reinterpret_cast<uintptr_t>(ptr);
@@ -506,21 +545,19 @@ int ltxattn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
   p.w[1] = static_cast<const __nv_bfloat16*>(k_weight);
   p.cos_t = cos_table;
   p.sin_t = sin_table;
-  p.rows = (long long)batch * seq_len;
+  if ((long long)batch * seq_len >= (1LL << 30)) return LTXATTN_ERR_UNSUPPORTED;
+  p.rows = batch * seq_len;
   p.seq_len = seq_len;
   p.head_dim = head_dim;
   p.eps = eps;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const long long blocks = (2 * p.rows + ltx::kPrologueWarps - 1) / ltx::kPrologueWarps;
-  if (blocks > 0x7fffffffLL) return LTXATTN_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)blocks), block(ltx::kPrologueWarps * 32);
   switch (inner) {
-    case 512: ltx::qk_norm_rope<2><<<grid, block, 0, stream>>>(p); break;
-    case 1024: ltx::qk_norm_rope<4><<<grid, block, 0, stream>>>(p); break;
-    case 2048: ltx::qk_norm_rope<8><<<grid, block, 0, stream>>>(p); break;
-    default: ltx::qk_norm_rope<16><<<grid, block, 0, stream>>>(p); break;
+    case 512: return launch_prologue<2, 1, 2>(p, stream);
+    case 1024: return launch_prologue<4, 1, 3>(p, stream);
+    case 2048: return launch_prologue<4, 2, 2>(p, stream);
+    case 4096: return launch_prologue<4, 4, 2>(p, stream);
+    default: return launch_prologue<4, 8, 3>(p, stream);
   }
-  return cudaGetLastError() == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
 int ltxattn_num_entry_points(void) {

@@ -40,6 +40,8 @@ SHAPES = [
     (3, 129, 32, 64),     # audio stream heads, inner 2048
     (2, 300, 32, 128),    # video stream heads, inner 4096
     (1, 50, 64, 64),      # inner 4096 with 64-channel heads
+    (2, 21, 64, 128),     # inner 8192: one row per CTA
+    (1, 9, 4, 256),       # inner 1024 with 256-channel heads
 ]
 
 
