@@ -23,6 +23,7 @@ numpy gathers and sums, no blocking or reordering beyond processing query rows i
 from __future__ import annotations
 
 import numpy as np
+import torch
 
 
 def window_start(i: np.ndarray, k: int, n: int) -> np.ndarray:
@@ -58,18 +59,19 @@ def na3d(q, k, v, grid, kernel, scale: float, rows=None, chunk: int = 2048) -> n
     Returns float64 [batch, len(rows), heads, head_dim] (all tokens when rows is None).
     """
     check_shape(grid, kernel)
-    qf, kf, vf = (t.double().numpy() for t in (q, k, v))
-    bsz, n_tok, heads, d = qf.shape
+    bsz, n_tok, heads, d = q.shape
     assert n_tok == grid[0] * grid[1] * grid[2], "sequence length = T * Y * X"
     rows = np.arange(n_tok) if rows is None else np.asarray(rows, dtype=np.int64)
     out = np.empty((bsz, len(rows), heads, d))
     for lo in range(0, len(rows), chunk):
         r = rows[lo:lo + chunk]
         idx = neighbours(r, grid, kernel)                      # [R, K]
+        rt, it = torch.from_numpy(r), torch.from_numpy(idx)
         for b in range(bsz):
-            qs = qf[b, r]                                      # [R, H, D]
-            ks = kf[b][idx]                                    # [R, K, H, D]
-            vs = vf[b][idx]
+            # only the rows this chunk needs are widened to float64
+            qs = q[b][rt].double().numpy()                     # [R, H, D]
+            ks = k[b][it].double().numpy()                     # [R, K, H, D]
+            vs = v[b][it].double().numpy()
             s = np.einsum("rhd,rkhd->rhk", qs, ks) * scale     # [R, H, K]
             s = s - s.max(axis=2, keepdims=True)
             p = np.exp(s)
