@@ -177,6 +177,35 @@ LTXATTN_API int ltxattn_qk_norm_rope(const void* q, const void* k, void* q_out, 
                                      int seq_len, int heads, int head_dim, float eps,
                                      ltxattn_stream_t stream);
 
+/*
+ * 3-D neighbourhood attention forward.  The LTX-2.5 diffusion decoder's stages attend
+ * over 3-D neighbourhoods (NATTEN's fused na3d; "LTX2.5", SGLang Diffusion cookbook, §4.6
+ * Diffusion decoder); the page gives no grid or window, and this call computes
+ * Neighborhood Attention's definition in three dimensions, without dilation and not
+ * causal.  Tokens sit on a grid_t x grid_y x grid_x grid in raster order, token
+ * n = (t * grid_y + y) * grid_x + x.  Along an axis of length N with window k, the query
+ * at position i sees the k positions starting at s(i) = min(max(i - (k-1)/2, 0), N - k)
+ * (centred, shifted inward at the borders); a query attends to the box of its three
+ * windows:
+ *     out[b,n,h,:] = sum_{m in box(n)} softmax_m(scale * q[b,n,h,:] . k[b,m,h,:]) v[b,m,h,:]
+ *
+ *   q, k, v, out  bf16 [batch, grid_t * grid_y * grid_x, heads, head_dim], contiguous
+ *                 (device); out must not overlap q, k or v
+ *   window_*      odd, 1 <= window <= its grid axis (INVALID_ARG otherwise)
+ *   head_dim      64 or 128 (UNSUPPORTED otherwise)
+ *   grid_t * grid_y * grid_x <= LTXATTN_MAX_LEN; heads, batch as for ltxattn_forward
+ *   scale         finite, > 0
+ * Precision as ltxattn_forward: bf16 products, fp32 scores and statistics, P rounded to
+ * bf16 before the PV product, output rounded to bf16.  Needs ltxattn_create on the
+ * current device.  Pointers 16-byte aligned (MISALIGNED).  Host checks run before any
+ * CUDA call; LTXATTN_ERR_CUDA on a failed launch; a kernel wait that times out is
+ * reported by ltxattn_check.  Asynchronous on `stream`.
+ */
+LTXATTN_API int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
+                                     int batch, int grid_t, int grid_y, int grid_x, int heads,
+                                     int head_dim, int window_t, int window_y, int window_x,
+                                     float scale, ltxattn_stream_t stream);
+
 /* Size of the library's built-in scratch array used by ltxattn_forward_split_noalloc. */
 #define LTXATTN_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per GPU */
 

@@ -17,6 +17,7 @@
 #include "fmha_fwd.cuh"
 #include "fmha_fwd_pp.cuh"
 #include "fmha_fwd_skv.cuh"
+#include "na3d_fwd.cuh"
 #include "qk_prologue.cuh"
 
 namespace {
@@ -54,7 +55,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_create",        "ltxattn_forward",          "ltxattn_forward_ex",
     "ltxattn_check",         "ltxattn_destroy",          "ltxattn_status_string",
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
-    "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope",
+    "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope", "ltxattn_na3d_forward",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -317,6 +318,73 @@ int launch_prologue(const ltx::PrologueParams& p, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- neighbourhood attention
+// Query brick shapes (t x y x x = 128 tokens) the kernel is built for; the host takes the
+// one whose bricks meet the fewest key tiles in total.
+struct NaShape {
+  int bt, by, bx;
+};
+constexpr NaShape kNaShapes[] = {{2, 8, 8}, {1, 8, 16}, {4, 4, 8}};
+
+template <int D, int BT, int BY, int BX>
+cudaError_t na_set_smem() {
+  return cudaFuncSetAttribute(ltx::na3d_fwd_sm100<D, BT, BY, BX>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, ltx::NaSmem<D>::kAlloc);
+}
+
+cudaError_t set_smem_limits_na() {
+  cudaError_t e = cudaSuccess;
+  for (cudaError_t x : {na_set_smem<64, 2, 8, 8>(), na_set_smem<64, 1, 8, 16>(),
+                        na_set_smem<64, 4, 4, 8>(), na_set_smem<128, 2, 8, 8>(),
+                        na_set_smem<128, 1, 8, 16>(), na_set_smem<128, 4, 4, 8>()})
+    if (x != cudaSuccess) e = x;
+  return e;
+}
+
+// Key tiles met by all query bricks of one (batch, head): per axis the sum over bricks of
+// the tiles covering their windows; the axes multiply.
+long long na_tiles_total(const NaShape& b, int t, int y, int x, int kt, int ky, int kx) {
+  auto axis = [](int n, int blk, int k) {
+    long long sum = 0;
+    for (int a0 = 0; a0 < n; a0 += blk) {
+      int r0, tiles;
+      ltx::na_key_span(a0, blk, k, n, r0, tiles);
+      sum += tiles;
+    }
+    return sum;
+  };
+  return axis(t, b.bt, kt) * axis(y, b.by, ky) * axis(x, b.bx, kx);
+}
+
+// BSHD bf16 tensor over a T x Y x X grid, [batch, T*Y*X, heads, head_dim], seen as a 5-D
+// TMA tensor (heads*head_dim, x, y, t, batch): a box is 64 columns of one head over a
+// bt x by x bx brick of tokens, 128-byte swizzled.
+bool encode_grid(const Context& c, CUtensorMap* map, const void* base, int batch, int t, int y,
+                 int x, int heads, int head_dim, const NaShape& b) {
+  const cuuint64_t row = (cuuint64_t)heads * head_dim * 2;
+  const cuuint64_t dims[5] = {(cuuint64_t)heads * head_dim, (cuuint64_t)x, (cuuint64_t)y,
+                              (cuuint64_t)t, (cuuint64_t)batch};
+  const cuuint64_t strides[4] = {row, row * x, row * x * y, row * x * y * t};
+  const cuuint32_t box[5] = {64, (cuuint32_t)b.bx, (cuuint32_t)b.by, (cuuint32_t)b.bt, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapL2promotion promo =
+      head_dim * 2 >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+  return c.encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BT, int BY, int BX>
+cudaError_t launch_na(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const CUtensorMap& to, const ltx::Na3dParams& p, int num_sms,
+                      cudaStream_t stream) {
+  const long long total = (long long)p.batch * p.heads * p.bricks;
+  const int grid = (int)std::min<long long>(total, num_sms);
+  ltx::na3d_fwd_sm100<D, BT, BY, BX>
+      <<<grid, ltx::kNaThreads, ltx::NaSmem<D>::kAlloc, stream>>>(tq, tk, tv, to, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
@@ -345,6 +413,7 @@ int ltxattn_create(void) {
          set_smem_limits<64>() == cudaSuccess && set_smem_limits<128>() == cudaSuccess &&
          set_smem_limits_pp<64>() == cudaSuccess && set_smem_limits_pp<128>() == cudaSuccess &&
          set_smem_limits_skv() == cudaSuccess && set_smem_limits_dual() == cudaSuccess &&
+         set_smem_limits_na() == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
@@ -558,6 +627,80 @@ int ltxattn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
     case 4096: return launch_prologue<4, 4, 2>(p, stream);
     default: return launch_prologue<4, 8, 3>(p, stream);
   }
+}
+
+int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out, int batch,
+                         int grid_t, int grid_y, int grid_x, int heads, int head_dim,
+                         int window_t, int window_y, int window_x, float scale,
+                         ltxattn_stream_t stream_) {
+  if (!q || !k || !v || !out) return LTXATTN_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || grid_t < 1 || grid_y < 1 || grid_x < 1)
+    return LTXATTN_ERR_INVALID_ARG;
+  const int grid_dims[3] = {grid_t, grid_y, grid_x}, win[3] = {window_t, window_y, window_x};
+  for (int a = 0; a < 3; ++a)
+    if (win[a] < 1 || win[a] % 2 == 0 || win[a] > grid_dims[a]) return LTXATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return LTXATTN_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LTXATTN_ERR_UNSUPPORTED;
+  const long long tokens = (long long)grid_t * grid_y * grid_x;
+  if (tokens > LTXATTN_MAX_LEN || heads > LTXATTN_MAX_HEADS || batch > LTXATTN_MAX_BATCH)
+    return LTXATTN_ERR_UNSUPPORTED;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
+  if (mis & 15u) return LTXATTN_ERR_MISALIGNED;
+  const size_t bytes = (size_t)batch * tokens * heads * head_dim * 2;
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+      overlaps(out, bytes, v, bytes))
+    return LTXATTN_ERR_INVALID_ARG;
+  int st;
+  Context* c = current_context(&st);
+  if (!c) return st;
+
+  int best = 0;
+  long long best_tiles = -1;
+  for (int i = 0; i < (int)(sizeof(kNaShapes) / sizeof(kNaShapes[0])); ++i) {
+    const long long t = na_tiles_total(kNaShapes[i], grid_t, grid_y, grid_x, window_t, window_y,
+                                       window_x);
+    if (best_tiles < 0 || t < best_tiles) {
+      best_tiles = t;
+      best = i;
+    }
+  }
+  const NaShape& sh = kNaShapes[best];
+  ltx::Na3dParams p{};
+  p.batch = batch;
+  p.heads = heads;
+  p.grid_t = grid_t;
+  p.grid_y = grid_y;
+  p.grid_x = grid_x;
+  p.win_t = window_t;
+  p.win_y = window_y;
+  p.win_x = window_x;
+  p.nb_t = (grid_t + sh.bt - 1) / sh.bt;
+  p.nb_y = (grid_y + sh.by - 1) / sh.by;
+  p.nb_x = (grid_x + sh.bx - 1) / sh.bx;
+  p.bricks = p.nb_t * p.nb_y * p.nb_x;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = c->d_status;
+  p.timeout_ns = kDefaultTimeoutNs;
+
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_grid(*c, &tq, q, batch, grid_t, grid_y, grid_x, heads, head_dim, sh) ||
+      !encode_grid(*c, &tk, k, batch, grid_t, grid_y, grid_x, heads, head_dim, sh) ||
+      !encode_grid(*c, &tv, v, batch, grid_t, grid_y, grid_x, heads, head_dim, sh) ||
+      !encode_grid(*c, &to, out, batch, grid_t, grid_y, grid_x, heads, head_dim, sh))
+    return LTXATTN_ERR_CUDA;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  cudaError_t e;
+  if (head_dim == 64) {
+    e = best == 0   ? launch_na<64, 2, 8, 8>(tq, tk, tv, to, p, c->num_sms, stream)
+        : best == 1 ? launch_na<64, 1, 8, 16>(tq, tk, tv, to, p, c->num_sms, stream)
+                    : launch_na<64, 4, 4, 8>(tq, tk, tv, to, p, c->num_sms, stream);
+  } else {
+    e = best == 0   ? launch_na<128, 2, 8, 8>(tq, tk, tv, to, p, c->num_sms, stream)
+        : best == 1 ? launch_na<128, 1, 8, 16>(tq, tk, tv, to, p, c->num_sms, stream)
+                    : launch_na<128, 4, 4, 8>(tq, tk, tv, to, p, c->num_sms, stream);
+  }
+  return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
 int ltxattn_num_entry_points(void) {

@@ -51,6 +51,7 @@ def load() -> ctypes.CDLL:
             lib.ltxattn_num_entry_points.argtypes = []
             lib.ltxattn_qk_norm_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                                  cf, vp]
+            lib.ltxattn_na3d_forward.argtypes = [vp, vp, vp, vp] + [ci] * 9 + [cf, vp]
             lib.ltxattn_entry_point_name.argtypes = [ci]
             lib.ltxattn_entry_point_name.restype = ctypes.c_char_p
             _lib = lib
@@ -196,3 +197,37 @@ def qk_norm_rope(q, k, q_weight, k_weight, cos, sin, q_out=None, k_out=None, *,
         ctypes.c_void_p(_stream_handle(stream)))
     _check(st, "ltxattn_qk_norm_rope")
     return q_out, k_out
+
+
+def na3d_forward(q, k, v, grid, window, out=None, *, scale: float | None = None, stream=None):
+    """3-D neighbourhood attention (``ltxattn_na3d_forward``) of bf16 CUDA tensors.
+
+    q, k, v: [B, T*Y*X, H, D] with tokens in raster order of the grid (T, Y, X); window
+    (kT, kY, kX): odd sizes, each at most its grid axis.  Returns out [B, T*Y*X, H, D].
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError(f"{name} must be a contiguous [batch, tokens, heads, head_dim] "
+                             "tensor shaped like q")
+    grid_t, grid_y, grid_x = (int(x) for x in grid)
+    win_t, win_y, win_x = (int(x) for x in window)
+    batch, tokens, heads, head_dim = q.shape
+    if tokens != grid_t * grid_y * grid_x:
+        raise ValueError(f"{tokens} tokens but grid {tuple(grid)}")
+    if out is None:
+        out = torch.empty_like(q)
+    elif (out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous()
+          or out.device != q.device):
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q on q's device")
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    st = load().ltxattn_na3d_forward(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()), int(batch), grid_t,
+        grid_y, grid_x, int(heads), int(head_dim), win_t, win_y, win_x, ctypes.c_float(scale),
+        ctypes.c_void_p(_stream_handle(stream)))
+    _check(st, "ltxattn_na3d_forward")
+    return out
