@@ -8,6 +8,7 @@ run back to back on one stream through the C ABI (libltxattn.so).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...     # the fp64 CPU oracle, timed on a sample
     python bench.py --workload qk_prologue   # the QK-norm + rotary prologue alone (GB/s)
+    python bench.py --workload na3d_decoder  # 3-D neighbourhood attention, decoder-size grid
 
 Prints one JSON line (rank 0).  ``value`` is the whole-job TFLOP/s (algorithmic
 FLOPs of all ranks / max-over-ranks device time); the timed region holds exactly
@@ -624,6 +625,145 @@ def run_prologue(args):
         dist.destroy_process_group()
 
 
+NA_SHAPES = ((2, 8, 8), (1, 8, 16), (4, 4, 8))  # query bricks the library is built for
+
+
+def na_key_tiles(grid, window):
+    """128-key tiles the neighbourhood kernel multiplies per (batch, head): the brick
+    shape with the fewest, as the library picks it (counting only; no attention math)."""
+    def start(i, k, n):
+        return min(max(i - k // 2, 0), n - k)
+
+    def axis(n, blk, k):
+        tot = 0
+        for a0 in range(0, n, blk):
+            a1 = min(a0 + blk, n)
+            r0, r1 = start(a0, k, n), start(a1 - 1, k, n) + k
+            tot += -(-(r1 - r0) // blk)
+        return tot
+
+    return min(axis(grid[0], sh[0], window[0]) * axis(grid[1], sh[1], window[1])
+               * axis(grid[2], sh[2], window[2]) for sh in NA_SHAPES)
+
+
+def run_na3d(args):
+    """3-D neighbourhood attention over the decoder-size grid (tensor-core kernel)."""
+    import torch
+
+    from joint_audio_video_flash_b200 import build, ltxattn, synth
+    world, rank, local = dist_setup(args.gpus)
+    build.build()
+    ltxattn.create()
+    grid, window, heads, d, b = (16, 34, 60), (3, 7, 7), 32, 128, 1
+    n = grid[0] * grid[1] * grid[2]
+    vol = window[0] * window[1] * window[2]
+    q, k, v = synth.make_qkv(b, n, n, heads, d, seed=77)
+    dev = torch.device("cuda", local)
+    dq, dk, dv = (t.to(dev) for t in (q, k, v))
+    out = torch.empty_like(dq)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ltxattn.na3d_forward(dq, dk, dv, grid, window, out)
+
+    if args.once:  # one launch, no timing: the command the Nsight Compute captures run
+        step()
+        torch.cuda.synchronize()
+        ltxattn.check()
+        print(json.dumps({"workload": args.workload, "once": True}))
+        return
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    ltxattn.check()
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ltxattn.check()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    # algorithmic work: every query against its neighbourhood (QK and PV, 2 FLOP a MAC)
+    step_flops = 4.0 * b * heads * n * vol * d
+    value = whole_job_tflops(step_flops, args.steps, world, total_ms)
+    tiles = na_key_tiles(grid, window) * b * heads
+    issued = tiles * 4.0 * 128 * 128 * d  # the 128 x 128 tiles the tensor cores multiply
+    issued_tflops = whole_job_tflops(issued, args.steps, world, total_ms)
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # end to end: q, k, v up from pinned host memory and the output down, every step
+    hq, hk, hv = (t.pin_memory() for t in (q, k, v))
+    hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ltxattn.check()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    line = {
+        "metric": "3-D neighbourhood attention TFLOP/s (neighbourhood FLOPs)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "na3d_decoder",
+                   "description": "grid 16 x 34 x 60 tokens (960x544x121 at 16x16 patches and "
+                                  "8-frame compression, a reading), window 3 x 7 x 7, "
+                                  "32 heads x 128, batch 1",
+                   "l2": "inputs larger than L2 (q, k, v 267 MB each)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "achieved": value, "peak": burst, "unit": "TFLOP/s",
+                     "frac": value / burst, "traffic": None,
+                     "kernel": "na3d_fwd_sm100<128, 2, 8, 8>",
+                     "issued_tflops": issued_tflops, "issued_frac": issued_tflops / burst,
+                     "density": step_flops / issued,
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "e2e": {"value": whole_job_tflops(step_flops, e2e_steps, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": q.numel() * 2,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import numpy as np
+
+        from oracle import na3d as na
+        done, secs, chunk = 0, 0.0, 512
+        while secs < args.cpu_seconds and done < n:
+            rows = np.arange(done, min(n, done + chunk))
+            t_start = time.perf_counter()
+            na.na3d(q, k, v, grid, window, d ** -0.5, rows=rows)
+            secs += time.perf_counter() - t_start
+            done += len(rows)
+        line["cpu_baseline"] = {"value": step_flops * (done / n) / secs / 1e12, "unit": "TFLOP/s",
+                                "cores": 1, "kind": "oracle",
+                                "sample": f"tokens 0..{done - 1} of {n}, all 32 heads; numpy "
+                                          f"fp64, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -640,6 +780,8 @@ def main():
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.workload == "qk_prologue" and args.impl != "reference":
         run_prologue(args)
+    elif args.workload == "na3d_decoder" and args.impl != "reference":
+        run_na3d(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

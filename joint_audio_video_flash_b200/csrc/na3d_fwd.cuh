@@ -14,7 +14,10 @@
 // union of their windows); it is covered by key tiles that are bricks of the same shape
 // starting at the box's corner (one 5-D TMA box each, zero fill past the grid), so a
 // query brick meets nt * ny * nx key tiles.  The scores of every tile are masked per
-// element against the query row's own window (three bit masks, one per axis).
+// element against the query row's own window (a bias of 0 or -inf per key column and per
+// (t, y) row of the tile, from three bit masks, one per axis), and a warp skips the
+// exponentials of each 32-key chunk that lies outside all of its rows' windows.
+// Softmax and epilogue warps arrive on their mbarriers once per warp, after __syncwarp.
 //
 // Persistent: one CTA per SM walks a contiguous run of (batch, head, brick) units:
 //   warp 0      TMA producer: Q bricks (2 stages, the next brick's Q issued with the
@@ -192,10 +195,10 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::bSF + s), 1);
-      mbar_init(bar(L::bPF + s), kBlockM);
+      mbar_init(bar(L::bPF + s), 4);
       mbar_init(bar(L::bOF + s), 1);
-      mbar_init(bar(L::bOE + s), kBlockM);
-      mbar_init(bar(L::bLF + s), kBlockM);
+      mbar_init(bar(L::bOE + s), 4);
+      mbar_init(bar(L::bLF + s), 4);
     }
     mbar_init(bar(L::bOD), 1);
     mbar_init(bar(L::bDrain), 1);
@@ -401,17 +404,29 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         const uint32_t mt = na_bits(wt0 - kt, wt0 - kt + p.win_t, BT);
         const uint32_t my = na_bits(wy0 - ky, wy0 - ky + p.win_y, BY);
         const uint32_t mx = na_bits(wx0 - kx, wx0 - kx + p.win_x, BX);
+        // window mask as additive biases (0 inside, -inf outside): one per key column x
+        // of the tile and one per (t, y) row of it, two packed adds per pair of scores
+        float2 bx2[BX / 2];
+#pragma unroll
+        for (int c2 = 0; c2 < BX / 2; ++c2)
+          bx2[c2] = make_float2((mx >> (2 * c2)) & 1u ? 0.0f : -INFINITY,
+                                (mx >> (2 * c2 + 1)) & 1u ? 0.0f : -INFINITY);
+        uint32_t rows_in = 0;  // (t, y) rows of the tile inside this query's window
         tmem_ld_wait();
 #pragma unroll
-        for (int a = 0; a < BT; ++a)
+        for (int r = 0; r < BT * BY; ++r) {
+          const bool in = (mt >> (r / BY)) & (my >> (r % BY)) & 1u;
+          rows_in |= (in ? 1u : 0u) << r;
+          const float rb = in ? 0.0f : -INFINITY;
+          const float2 rb2 = make_float2(rb, rb);
 #pragma unroll
-          for (int bb = 0; bb < BY; ++bb) {
-            // keys (a, bb, 0 .. BX) of the tile: the x mask where the (t, y) pair is in
-            const uint32_t mrow = ((mt >> a) & (my >> bb) & 1u) ? mx : 0u;
-#pragma unroll
-            for (int cc = 0; cc < BX; ++cc)
-              if (!((mrow >> cc) & 1u)) s[(a * BY + bb) * BX + cc] = -INFINITY;
+          for (int c2 = 0; c2 < BX / 2; ++c2) {
+            float2 v = make_float2(s[r * BX + 2 * c2], s[r * BX + 2 * c2 + 1]);
+            v = __fadd2_rn(__fadd2_rn(v, bx2[c2]), rb2);
+            s[r * BX + 2 * c2] = v.x;
+            s[r * BX + 2 * c2 + 1] = v.y;
           }
+        }
         const float mx_t = row_max<kBlockN>(s) * sl2;
         const bool grow = m_run != -INFINITY && mx_t > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, grow)) {
@@ -441,15 +456,26 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         const float m_use = m_run == -INFINITY ? 0.0f : m_run;
         const float2 nm2 = make_float2(-m_use, -m_use);
         float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
+        if (mx == 0) rows_in = 0;
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
+          // a 32-key chunk outside every window of this warp's rows: P = 0 without the
+          // exponentials (the MUFU bounds this loop)
+          constexpr int kRowsChunk = 32 / BX;
+          const uint32_t chunk_rows = (rows_in >> (c * kRowsChunk)) & ((1u << kRowsChunk) - 1u);
           uint32_t pk[16];
-          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+          if (__any_sync(0xffffffffu, chunk_rows != 0)) {
+            exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) pk[x] = 0u;
+          }
           tmem_st16(tS + c * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::bPF + sb));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::bPF + sb));
         l_run += (la.x + la.y) + (lb.x + lb.y);
       }
       if (!ok) break;
@@ -459,7 +485,8 @@ __global__ void __launch_bounds__(kNaThreads, 1)
                         mbar_wait(bar(L::bOE + ob), (uint32_t)((i >> 1) - 1) & 1u, ctl));
       if (!ok) break;
       row_sum[ob * kBlockM + row] = l_run;
-      mbar_arrive(bar(L::bLF + ob));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::bLF + ob));
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -495,7 +522,8 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         tmem_ld_wait();
         if (bx == L::kBoxes - 1) {
           tc_fence_before();
-          mbar_arrive(bar(L::bOE + ob));  // O buffer and row sums of brick i are read
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(L::bOE + ob));
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
