@@ -61,3 +61,21 @@ def test_gpu_arm_line():
     assert set(d["per_call"]) == {"video_self", "audio_self", "v2a", "a2v"}
     assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("workload,unit", [("na3d_decoder", "TFLOP/s"), ("qk_prologue", "GB/s")])
+def test_gpu_arm_line_other_workloads(workload, unit):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    d = _run(["--workload", workload, "--steps", "3", "--warmup", "3", "--cpu-seconds", "1"],
+             timeout=900)
+    assert COMMON <= set(d) and "impl" not in d
+    assert d["unit"] == unit and d["value"] > 0 and d["config"]["workload"] == workload
+    r = d["roofline"]
+    assert r["achieved"] > 0 and r["peak"] > 0 and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    e = d["e2e"]
+    assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
+    assert d["gpu_launches"] == d["steps"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
