@@ -36,14 +36,23 @@ METRIC = "attention TFLOP/s and µs/call per config; % of B200 dense-BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, keyed by
-# the hash of the kernel sources it was taken on; reported as null once the sources change.
+# the hash of the sources that make up that kernel; reported as null once they change.
+KERNEL_SOURCES = {
+    "video_self": ("joint_audio_video_flash_b200/csrc/fmha_fwd_pp.cuh",
+                   "joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
+                   "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
+    "na3d_decoder": ("joint_audio_video_flash_b200/csrc/na3d_fwd.cuh",
+                     "joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
+                     "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
+    "qk_prologue": ("joint_audio_video_flash_b200/csrc/qk_prologue.cuh",
+                    "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
+}
 TRAFFIC = {
     "video_self": {"src": "3fe5540a7028fb95", "bytes_per_token": (201.515264e6 + 46.888448e6) / 8192,
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
+    "na3d_decoder": {"src": "7dc0842a39a1e72a", "bytes": 951.997696e6 + 253.550848e6,
+                     "note": "full launch, 16x34x60 grid, 3x7x7 window, 32x128"},
 }
-KERNEL_SOURCES = ("joint_audio_video_flash_b200/csrc/fmha_fwd_pp.cuh",
-                  "joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
-                  "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh")
 
 
 def kernel_label(c, num_sms: int = 148) -> str:
@@ -59,13 +68,21 @@ def kernel_label(c, num_sms: int = 148) -> str:
     return f"fmha_fwd_sm100<{c.head_dim}>"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str = "video_self") -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def traffic_per_launch(kernel: str):
+    """ncu DRAM bytes per launch of `kernel`, or None when its sources changed since."""
+    tr = TRAFFIC.get(kernel)
+    if tr is None or tr["src"] != kernel_source_hash(kernel):
+        return None
+    return tr.get("bytes")
 
 
 def load_peaks():
@@ -430,7 +447,7 @@ def run_ltxattn(args):
     tflops_peak = burst if at_max else sustained
     tr = TRAFFIC.get(calls[vi].name)
     traffic = None
-    if tr is not None and tr["src"] == kernel_source_hash():
+    if tr is not None and tr["src"] == kernel_source_hash("video_self"):
         traffic = tr["bytes_per_token"] * calls[vi].batch * calls[vi].q_len
     if calls[vi].flops / calls[vi].bytes > tflops_peak * 1e12 / (hbm * 1e9):
         achieved = calls[vi].flops / (v_us * 1e-6) / 1e12
@@ -595,7 +612,8 @@ def run_prologue(args):
                    "l2": "inputs larger than L2 (q and k are 252 MB each)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": value, "peak": hbm, "unit": "GB/s",
-                     "frac": value / hbm, "traffic": None, "kernel": "qk_norm_rope<4, 4, 2>",
+                     "frac": value / hbm, "traffic": traffic_per_launch("qk_prologue"),
+                     "kernel": "qk_norm_rope<4, 4, 2>",
                      "algorithmic_bytes": step_bytes, "peak_source": f"{peak_src} hbm_gbs"},
         "e2e": {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": 2 * q.numel() * 2, "d2h_bytes_per_step": 2 * q.numel() * 2},
@@ -731,7 +749,7 @@ def run_na3d(args):
                    "l2": "inputs larger than L2 (q, k, v 267 MB each)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "achieved": value, "peak": burst, "unit": "TFLOP/s",
-                     "frac": value / burst, "traffic": None,
+                     "frac": value / burst, "traffic": traffic_per_launch("na3d_decoder"),
                      "kernel": "na3d_fwd_sm100<128, 2, 8, 8>",
                      "issued_tflops": issued_tflops, "issued_frac": issued_tflops / burst,
                      "density": step_flops / issued,
