@@ -43,6 +43,11 @@ CASES = [
     (2, (1, 24, 40), 2, 64, (1, 7, 9)),    # 1x8x16, a 2-D grid
     (1, (16, 8, 8), 1, 128, (7, 3, 3)),    # 2x8x8, long time axis
     (1, (12, 6, 9), 2, 64, (5, 3, 5)),     # 2x8x8, bricks wider than the grid
+    (2, (1, 8, 8), 2, 128, (1, 3, 3)),     # 2x8x8 on a one-frame grid: half of each brick is past it
+    (1, (1, 5, 6), 1, 64, (1, 3, 5)),      # a grid smaller than one brick on every axis
+    (2, (3, 10, 13), 2, 128, (3, 5, 7)),   # 4x4x8 at head_dim 128, batch 2
+    (1, (9, 4, 5), 3, 128, (5, 3, 3)),     # 4x4x8, three heads, long time axis
+    (1, (2, 3, 40), 2, 64, (1, 3, 9)),     # 2x8x8, long thin grid
 ]
 
 
