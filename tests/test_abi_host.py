@@ -91,3 +91,61 @@ def test_valid_arguments_reach_cuda(lib):
     assert lib.ltxattn_create() == ltxattn.ERR_CUDA
     assert lib.ltxattn_selftest_wait_timeout(ctypes.c_ulonglong(10), None) == \
         ltxattn.ERR_INVALID_ARG
+
+
+def na3d(lib, q=Q, k=K, v=V, o=O, batch=1, grid=(2, 8, 8), heads=2, d=64, win=(1, 3, 3),
+         scale=0.125):
+    return lib.ltxattn_na3d_forward(ctypes.c_void_p(q), ctypes.c_void_p(k), ctypes.c_void_p(v),
+                                    ctypes.c_void_p(o), batch, *grid, heads, d, *win,
+                                    ctypes.c_float(scale), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(v=0), ltxattn.ERR_INVALID_ARG),
+    (dict(batch=0), ltxattn.ERR_INVALID_ARG),
+    (dict(grid=(0, 8, 8)), ltxattn.ERR_INVALID_ARG),
+    (dict(win=(2, 3, 3)), ltxattn.ERR_INVALID_ARG),       # even window
+    (dict(win=(1, 3, 0)), ltxattn.ERR_INVALID_ARG),
+    (dict(win=(3, 3, 3)), ltxattn.ERR_INVALID_ARG),       # window longer than its axis (t = 2)
+    (dict(win=(1, 9, 3)), ltxattn.ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ltxattn.ERR_INVALID_ARG),
+    (dict(d=96), ltxattn.ERR_UNSUPPORTED),
+    (dict(grid=(2, 1 << 12, 1 << 12)), ltxattn.ERR_UNSUPPORTED),  # 2^25 tokens
+    (dict(heads=1025), ltxattn.ERR_UNSUPPORTED),
+    (dict(k=K + 8), ltxattn.ERR_MISALIGNED),
+    (dict(o=V + 64), ltxattn.ERR_INVALID_ARG),             # out overlaps v
+])
+def test_na3d_host_validation(lib, kw, status):
+    assert na3d(lib, **kw) == status
+
+
+def qk(lib, q=Q, k=K, qo=O, ko=O + (1 << 20), wq=9 << 20, wk=10 << 20, cos=11 << 20,
+       sin=12 << 20, batch=1, seq=16, heads=8, d=128, eps=1e-6):
+    return lib.ltxattn_qk_norm_rope(*(ctypes.c_void_p(x) for x in (q, k, qo, ko, wq, wk)),
+                                    ctypes.c_void_p(cos), ctypes.c_void_p(sin), batch, seq,
+                                    heads, d, ctypes.c_float(eps), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(wq=0), ltxattn.ERR_INVALID_ARG),
+    (dict(seq=0), ltxattn.ERR_INVALID_ARG),
+    (dict(eps=-1.0), ltxattn.ERR_INVALID_ARG),
+    (dict(eps=float("inf")), ltxattn.ERR_INVALID_ARG),
+    (dict(heads=3, d=64), ltxattn.ERR_UNSUPPORTED),        # inner 192
+    (dict(heads=4, d=36), ltxattn.ERR_UNSUPPORTED),        # head_dim not a multiple of 8
+    (dict(heads=128, d=128), ltxattn.ERR_UNSUPPORTED),     # inner 16384
+    (dict(cos=(11 << 20) + 4), ltxattn.ERR_MISALIGNED),
+    (dict(ko=Q), ltxattn.ERR_INVALID_ARG),                 # k_out overlaps q
+    (dict(qo=K), ltxattn.ERR_INVALID_ARG),                 # q_out overlaps k
+])
+def test_qk_norm_rope_host_validation(lib, kw, status):
+    assert qk(lib, **kw) == status
+
+
+def test_new_calls_reach_cuda_with_valid_arguments(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-only expectation: no CUDA device")
+    assert na3d(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
+    assert qk(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
+    assert qk(lib, qo=Q, ko=K) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)  # in place
