@@ -505,6 +505,122 @@ def run_ltxattn(args):
         dist.destroy_process_group()
 
 
+PROLOGUE_SHAPE, PROLOGUE_SEED = (2, 15360, 32, 128), 21  # batch, tokens, heads, head_dim
+PROLOGUE_METRIC = "qk norm + rotary prologue GB/s"
+NA_GRID, NA_WINDOW, NA_HEADS, NA_D, NA_BATCH, NA_SEED = (16, 34, 60), (3, 7, 7), 32, 128, 1, 77
+NA_METRIC = "3-D neighbourhood attention TFLOP/s (neighbourhood FLOPs)"
+
+
+def prologue_config(world):
+    return {"workload": "qk_prologue",
+            "description": "queries and keys of the video stream, B2 x 15360 tokens x "
+                           "32 heads x 128: RMSNorm over heads*dim, rotary on channel "
+                           "pairs (a reading; see the header)",
+            "l2": "inputs larger than L2 (q and k are 252 MB each)",
+            "parallelism": f"replicas x{world}"}
+
+
+def prologue_step_bytes():
+    b, l, h, d = PROLOGUE_SHAPE
+    # q and k read and written once (bf16); weights and tables are 0.1 %
+    return 4.0 * b * l * h * d * 2 + 2 * h * d * 2 + 2 * l * (d // 2) * 4
+
+
+def prologue_oracle_time(inputs, seconds, start=0, block=512):
+    """Runs the fp64 oracle over token blocks from `start` for about `seconds`; returns
+    (tokens done, seconds)."""
+    from oracle import qk_prologue as qp
+    q, k, wq, wk, cos, sin = inputs
+    l = q.shape[1]
+    done, secs = 0, 0.0
+    while done < l and secs < seconds:
+        a = (start + done) % l
+        sl = slice(a, min(l, a + block))
+        t_start = time.perf_counter()
+        qp.rms_norm_rope(q[:, sl], wq, cos[sl], sin[sl], 1e-6)
+        qp.rms_norm_rope(k[:, sl], wk, cos[sl], sin[sl], 1e-6)
+        secs += time.perf_counter() - t_start
+        done += sl.stop - sl.start
+    return done, secs
+
+
+def na3d_config(world):
+    return {"workload": "na3d_decoder",
+            "description": "grid 16 x 34 x 60 tokens (960x544x121 at 16x16 patches and "
+                           "8-frame compression, a reading), window 3 x 7 x 7, "
+                           "32 heads x 128, batch 1",
+            "l2": "inputs larger than L2 (q, k, v 267 MB each)",
+            "parallelism": f"replicas x{world}"}
+
+
+def na3d_step_flops():
+    n = NA_GRID[0] * NA_GRID[1] * NA_GRID[2]
+    vol = NA_WINDOW[0] * NA_WINDOW[1] * NA_WINDOW[2]
+    # every query against its neighbourhood: QK and PV, 2 FLOP a multiply-add
+    return 4.0 * NA_BATCH * NA_HEADS * n * vol * NA_D
+
+
+def na3d_oracle_time(q, k, v, seconds, start=0, chunk=512):
+    """Runs the fp64 oracle over query-token chunks from `start` for about `seconds`;
+    returns (tokens done, seconds)."""
+    import numpy as np
+
+    from oracle import na3d as na
+    n = q.shape[1]
+    done, secs = 0, 0.0
+    while secs < seconds and done < n:
+        a = (start + done) % n
+        rows = np.arange(a, min(n, a + chunk))
+        t_start = time.perf_counter()
+        na.na3d(q, k, v, NA_GRID, NA_WINDOW, NA_D ** -0.5, rows=rows)
+        secs += time.perf_counter() - t_start
+        done += len(rows)
+    return done, secs
+
+
+def run_reference_other(args):
+    """Reference arm of the prologue and neighbourhood workloads: their fp64 oracles, timed
+    on a bounded sample per step (CPU only; rank 0 alone)."""
+    from joint_audio_video_flash_b200 import synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    per_step_s = max(1.0, args.reference_budget_s / (args.steps + args.warmup))
+    if args.workload == "qk_prologue":
+        b, l, h, d = PROLOGUE_SHAPE
+        inputs = synth.make_qk_prologue_inputs(b, l, h, d, seed=PROLOGUE_SEED)
+        run = lambda st: prologue_oracle_time(inputs, per_step_s, start=st * 4096)  # noqa: E731
+        total, per_token, metric, unit, config = l, prologue_step_bytes() / l / 1e9, \
+            PROLOGUE_METRIC, "GB/s", prologue_config(world)
+        what = "token blocks of 512, both batch elements, q and k; numpy fp64, one core"
+    else:
+        n = NA_GRID[0] * NA_GRID[1] * NA_GRID[2]
+        q, k, v = synth.make_qkv(NA_BATCH, n, n, NA_HEADS, NA_D, seed=NA_SEED)
+        run = lambda st: na3d_oracle_time(q, k, v, per_step_s, start=st * 4096)  # noqa: E731
+        total, per_token, metric, unit, config = n, na3d_step_flops() / n / 1e12, \
+            NA_METRIC, "TFLOP/s", na3d_config(world)
+        what = "query-token chunks of 512, all 32 heads; numpy fp64, one core"
+    for w in range(args.warmup):
+        run(100 + w)
+    done = secs = 0.0
+    for st in range(args.steps):
+        a, b_ = run(st)
+        done += a
+        secs += b_
+    value = per_token * done / secs
+    sample = f"{int(done)} of {total} tokens per workload pass over {args.steps} steps: {what}"
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": unit,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_prologue(args):
     """The QK-norm + rotary prologue at the video stream's size (HBM-bound streaming kernel)."""
     import torch
@@ -512,8 +628,8 @@ def run_prologue(args):
     from joint_audio_video_flash_b200 import build, ltxattn, synth
     world, rank, local = dist_setup(args.gpus)
     build.build()
-    b, l, h, d = 2, 15360, 32, 128
-    q, k, wq, wk, cos, sin = synth.make_qk_prologue_inputs(b, l, h, d, seed=21)
+    b, l, h, d = PROLOGUE_SHAPE
+    q, k, wq, wk, cos, sin = synth.make_qk_prologue_inputs(b, l, h, d, seed=PROLOGUE_SEED)
     dev = torch.device("cuda", local)
     dq, dk, dwq, dwk, dcos, dsin = (t.to(dev) for t in (q, k, wq, wk, cos, sin))
     qo, ko = torch.empty_like(dq), torch.empty_like(dk)
@@ -545,8 +661,7 @@ def run_prologue(args):
         torch.cuda.synchronize()
         barrier(world)
     total_ms = max_over_ranks(t0.elapsed_time(t1), world)
-    # algorithmic bytes: q and k read and written once (bf16); weights and tables are 0.1 %
-    step_bytes = 4.0 * dq.numel() * 2 + 2 * dwq.numel() * 2 + 2 * dcos.numel() * 4
+    step_bytes = prologue_step_bytes()
     value = step_bytes * args.steps * world / (total_ms * 1e-3) / 1e9
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -603,16 +718,11 @@ def run_prologue(args):
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     line = {
-        "metric": "qk norm + rotary prologue GB/s", "value": value, "unit": "GB/s",
+        "metric": PROLOGUE_METRIC, "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "qk_prologue",
-                   "description": "queries and keys of the video stream, B2 x 15360 tokens x "
-                                  "32 heads x 128: RMSNorm over heads*dim, rotary on channel "
-                                  "pairs (a reading; see the header)",
-                   "l2": "inputs larger than L2 (q and k are 252 MB each)",
-                   "parallelism": f"replicas x{world}"},
+        "config": prologue_config(world),
         "roofline": {"bound": "hbm", "achieved": value, "peak": hbm, "unit": "GB/s",
                      "frac": value / hbm, "traffic": traffic_per_launch("qk_prologue"),
                      "kernel": "qk_norm_rope<4, 4, 2>",
@@ -624,19 +734,11 @@ def run_prologue(args):
     }
     line["e2e"]["steps"] = e2e_steps
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from oracle import qk_prologue as qp
-        blk, done, secs = 512, 0, 0.0
-        while done < l and secs < args.cpu_seconds:
-            sl = slice(done, min(l, done + blk))
-            t_start = time.perf_counter()
-            qp.rms_norm_rope(q[:, sl], wq, cos[sl], sin[sl], 1e-6)
-            qp.rms_norm_rope(k[:, sl], wk, cos[sl], sin[sl], 1e-6)
-            secs += time.perf_counter() - t_start
-            done = sl.stop
+        done, secs = prologue_oracle_time((q, k, wq, wk, cos, sin), args.cpu_seconds)
         line["cpu_baseline"] = {"value": step_bytes * (done / l) / secs / 1e9, "unit": "GB/s",
                                 "cores": 1, "kind": "oracle",
                                 "sample": f"token positions 0..{done - 1} of {l} in blocks of "
-                                          f"{blk}, both batch elements, q and k; numpy fp64, "
+                                          f"512, both batch elements, q and k; numpy fp64, "
                                           f"{secs:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -674,10 +776,9 @@ def run_na3d(args):
     world, rank, local = dist_setup(args.gpus)
     build.build()
     ltxattn.create()
-    grid, window, heads, d, b = (16, 34, 60), (3, 7, 7), 32, 128, 1
+    grid, window, heads, d, b = NA_GRID, NA_WINDOW, NA_HEADS, NA_D, NA_BATCH
     n = grid[0] * grid[1] * grid[2]
-    vol = window[0] * window[1] * window[2]
-    q, k, v = synth.make_qkv(b, n, n, heads, d, seed=77)
+    q, k, v = synth.make_qkv(b, n, n, heads, d, seed=NA_SEED)
     dev = torch.device("cuda", local)
     dq, dk, dv = (t.to(dev) for t in (q, k, v))
     out = torch.empty_like(dq)
@@ -712,8 +813,7 @@ def run_na3d(args):
         barrier(world)
     ltxattn.check()
     total_ms = max_over_ranks(t0.elapsed_time(t1), world)
-    # algorithmic work: every query against its neighbourhood (QK and PV, 2 FLOP a MAC)
-    step_flops = 4.0 * b * heads * n * vol * d
+    step_flops = na3d_step_flops()
     value = whole_job_tflops(step_flops, args.steps, world, total_ms)
     tiles = na_key_tiles(grid, window) * b * heads
     issued = tiles * 4.0 * 128 * 128 * d  # the 128 x 128 tiles the tensor cores multiply
@@ -740,16 +840,11 @@ def run_na3d(args):
     ltxattn.check()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     line = {
-        "metric": "3-D neighbourhood attention TFLOP/s (neighbourhood FLOPs)", "value": value,
+        "metric": NA_METRIC, "value": value,
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "na3d_decoder",
-                   "description": "grid 16 x 34 x 60 tokens (960x544x121 at 16x16 patches and "
-                                  "8-frame compression, a reading), window 3 x 7 x 7, "
-                                  "32 heads x 128, batch 1",
-                   "l2": "inputs larger than L2 (q, k, v 267 MB each)",
-                   "parallelism": f"replicas x{world}"},
+        "config": na3d_config(world),
         "roofline": {"bound": "tensor", "achieved": value, "peak": burst, "unit": "TFLOP/s",
                      "frac": value / burst, "traffic": traffic_per_launch("na3d_decoder"),
                      "kernel": "na3d_fwd_sm100<128, 2, 8, 8>",
@@ -763,16 +858,7 @@ def run_na3d(args):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import numpy as np
-
-        from oracle import na3d as na
-        done, secs, chunk = 0, 0.0, 512
-        while secs < args.cpu_seconds and done < n:
-            rows = np.arange(done, min(n, done + chunk))
-            t_start = time.perf_counter()
-            na.na3d(q, k, v, grid, window, d ** -0.5, rows=rows)
-            secs += time.perf_counter() - t_start
-            done += len(rows)
+        done, secs = na3d_oracle_time(q, k, v, args.cpu_seconds)
         line["cpu_baseline"] = {"value": step_flops * (done / n) / secs / 1e12, "unit": "TFLOP/s",
                                 "cores": 1, "kind": "oracle",
                                 "sample": f"tokens 0..{done - 1} of {n}, all 32 heads; numpy "
@@ -798,9 +884,11 @@ def main():
                     help="run each call of the workload once and exit (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
-    if args.workload == "qk_prologue" and args.impl != "reference":
+    if args.workload in ("qk_prologue", "na3d_decoder") and args.impl == "reference":
+        run_reference_other(args)
+    elif args.workload == "qk_prologue":
         run_prologue(args)
-    elif args.workload == "na3d_decoder" and args.impl != "reference":
+    elif args.workload == "na3d_decoder":
         run_na3d(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -41,6 +41,18 @@ def test_reference_arm_line():
                         "d2h_bytes_per_step": 0}
 
 
+@pytest.mark.parametrize("workload,unit", [("qk_prologue", "GB/s"), ("na3d_decoder", "TFLOP/s")])
+def test_reference_arm_line_other_workloads(workload, unit):
+    d = _run(["--impl", "reference", "--workload", workload, "--steps", "1", "--warmup", "0",
+              "--reference-budget-s", "2"], timeout=600)
+    assert COMMON <= set(d) and d["impl"] == "reference" and d["dtype"] == "f64"
+    assert d["unit"] == unit and d["value"] > 0 and d["config"]["workload"] == workload
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
 @pytest.mark.gpu
 def test_gpu_arm_line():
     import torch
