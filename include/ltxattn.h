@@ -206,6 +206,43 @@ LTXATTN_API int ltxattn_na3d_forward(const void* q, const void* k, const void* v
                                      int head_dim, int window_t, int window_y, int window_x,
                                      float scale, ltxattn_stream_t stream);
 
+/*
+ * Attention over one key range, left unnormalised across ranges: the building block of
+ * context-parallel attention, where each rank holds a shard of the keys and values and the
+ * ranks exchange per-range results in fp32 with their softmax statistics ("feat(ltx2):
+ * tile-parallel video VAE and the two-stage pipeline", commit "Onboard Lightricks LTX-2.5":
+ * CP over ranks with an fp32 statistics all-gather).  For every (b, h) and query row i:
+ *     o_part[b][h][i][:] = softmax_j(scale * q_i . k_j) v_j   over keys j < kv_valid_len
+ *     lse[b][h][i]       = log2 sum_{j < kv_valid_len} exp(scale * q_i . k_j)
+ * (base-2 log-sum-exp).  q, k, v as for ltxattn_forward (bf16 BSHD, device).
+ *
+ *   o_part  fp32 [batch][heads][rows_pad][head_dim] (device), rows_pad = ceil(q_len/128)*128;
+ *           rows i >= q_len are not written
+ *   lse     fp32 [batch][heads][rows_pad] (device)
+ * Same argument rules as ltxattn_forward (o_part takes out's place in the checks); neither
+ * output may overlap q, k, v or the other; 16-byte aligned.  Needs ltxattn_create.
+ * Asynchronous on `stream`; LTXATTN_ERR_CUDA on a failed launch.
+ */
+LTXATTN_API int ltxattn_forward_partial(const void* q, const void* k, const void* v, float* o_part,
+                                        float* lse, int q_len, int kv_len, int kv_valid_len,
+                                        int batch, int heads, int head_dim, float scale,
+                                        ltxattn_stream_t stream);
+
+/*
+ * Merge of `parts` results of ltxattn_forward_partial for the same queries over disjoint key
+ * ranges into the attention over their union (same statistics merge):
+ *     L = max_p lse_p,  w_p = 2^(lse_p - L),  out = sum_p w_p o_p / sum_p w_p   (fp32, then bf16)
+ *
+ *   o_parts  fp32 [parts][batch][heads][rows_pad][head_dim] (device), rows_pad as above
+ *   lses     fp32 [parts][batch][heads][rows_pad] (device)
+ *   out      bf16 [batch][q_len][heads][head_dim] (device), must not overlap the inputs
+ * head_dim 64 or 128; 1 <= parts <= 65536; 16-byte aligned pointers.  Needs no ltxattn_create.
+ * Asynchronous on `stream`.
+ */
+LTXATTN_API int ltxattn_combine(const float* o_parts, const float* lses, void* out, int parts,
+                                int q_len, int batch, int heads, int head_dim,
+                                ltxattn_stream_t stream);
+
 /* Size of the library's built-in scratch array used by ltxattn_forward_split_noalloc. */
 #define LTXATTN_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB per GPU */
 

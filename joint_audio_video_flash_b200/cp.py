@@ -1,0 +1,126 @@
+"""Context-parallel attention over the ranks of a process group (one process per GPU).
+
+The LTX-2.5 DiT splits the video sequence over context-parallel ranks, replicates the
+audio stream, and merges cross-attention results through an fp32 all-gather of per-rank
+softmax statistics ("feat(ltx2): tile-parallel video VAE and the two-stage pipeline",
+commit "Onboard Lightricks LTX-2.5"; "LTX-2: replicate audio stream across Ulysses ranks
+by default", Description).  Two exchange patterns cover the block's attentions:
+
+* self-attention over a sharded sequence (video self): every rank gathers all shards of K
+  and V, computes its own queries' attention over each shard as a partial result (fp32
+  output and base-2 log-sum-exp, ``ltxattn_forward_partial``) and merges the partials
+  (``ltxattn_combine``);
+* replicated queries over sharded keys and values (v2a: audio queries, video keys): every
+  rank computes the partial over its own shard; the partials and their statistics are
+  all-gathered and merged, so every rank ends with the full result.
+
+a2v (video queries over the replicated audio keys) and audio self-attention need no
+exchange: they run locally through ``ltxattn.forward``.
+
+Shards are contiguous, equal ranges of ceil(L / world) tokens, rank r holding tokens
+[r * Ls, min(L, (r + 1) * Ls)), zero-padded to Ls; a rank whose range is empty contributes
+no partial.  The collectives are torch.distributed all-gathers (NCCL between GPUs); every
+step of the attention itself runs in the library's kernels (``backend``, which tests on
+CPU replace).
+"""
+from __future__ import annotations
+
+import math
+
+
+class LibraryBackend:
+    """The library's kernels (CUDA tensors)."""
+
+    def partial(self, q, k, v, kv_valid_len, scale, o_part=None, lse=None):
+        from . import ltxattn
+        return ltxattn.forward_partial(q, k, v, o_part, lse, kv_valid_len=kv_valid_len,
+                                       scale=scale)
+
+    def combine(self, o_parts, lses, q_len):
+        from . import ltxattn
+        return ltxattn.combine(o_parts, lses, q_len)
+
+
+def shard_len(total: int, world: int) -> int:
+    """Tokens per shard (the last shard may hold fewer real tokens, or none)."""
+    return -(-int(total) // int(world))
+
+
+def shard_valid(total: int, world: int, rank: int) -> int:
+    """Real tokens in rank's shard."""
+    ls = shard_len(total, world)
+    return max(0, min(ls, int(total) - rank * ls))
+
+
+def _gather(t, group):
+    """[world, *t.shape] stack of every rank's t (rank order)."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    out = torch.empty((world, *t.shape), dtype=t.dtype, device=t.device)
+    dist.all_gather(list(out.unbind(0)), t.contiguous(), group=group)
+    return out
+
+
+def _rows_pad(q_len: int) -> int:
+    return -(-int(q_len) // 128) * 128
+
+
+def self_attention(q_local, k_local, v_local, seq_len: int, group, *, scale: float | None = None,
+                   backend=None):
+    """Attention of this rank's query shard over the whole sharded sequence.
+
+    q_local, k_local, v_local: [B, Ls, H, D], this rank's shard of a sequence of seq_len
+    tokens (zero-padded to Ls = ceil(seq_len / world)).  Returns [B, Ls, H, D]; rows past
+    the rank's real tokens are not meaningful.
+    """
+    import torch
+    import torch.distributed as dist
+    backend = backend or LibraryBackend()
+    world = dist.get_world_size(group)
+    batch, ls, heads, d = q_local.shape
+    if ls != shard_len(seq_len, world) or k_local.shape != q_local.shape or \
+            v_local.shape != q_local.shape:
+        raise ValueError(f"shards must be [B, {shard_len(seq_len, world)}, H, D] on every rank")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    kb, vb = _gather(k_local, group), _gather(v_local, group)
+    ranks = [r for r in range(world) if shard_valid(seq_len, world, r) > 0]
+    rp = _rows_pad(ls)
+    o_parts = torch.empty((len(ranks), batch, heads, rp, d), dtype=torch.float32,
+                          device=q_local.device)
+    lses = torch.empty((len(ranks), batch, heads, rp), dtype=torch.float32,
+                       device=q_local.device)
+    for i, r in enumerate(ranks):
+        backend.partial(q_local, kb[r], vb[r], shard_valid(seq_len, world, r), scale,
+                        o_parts[i], lses[i])
+    return backend.combine(o_parts, lses, ls)
+
+
+def cross_attention(q, k_local, v_local, kv_len: int, group, *, scale: float | None = None,
+                    backend=None):
+    """Replicated queries over keys and values sharded across the ranks (v2a).
+
+    q: [B, Lq, H, D], the same on every rank; k_local, v_local: [B, Ls, H, D], this rank's
+    shard of kv_len tokens.  Every rank returns the full result [B, Lq, H, D].
+    """
+    import torch.distributed as dist
+    backend = backend or LibraryBackend()
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    ls = shard_len(kv_len, world)
+    if k_local.shape[1] != ls or v_local.shape != k_local.shape:
+        raise ValueError(f"key/value shards must hold {ls} tokens on every rank")
+    scale = 1.0 / math.sqrt(q.shape[3]) if scale is None else scale
+    valid = shard_valid(kv_len, world, rank)
+    if valid > 0:
+        o_part, lse = backend.partial(q, k_local, v_local, valid, scale)
+    else:
+        import torch
+        batch, q_len, heads, d = q.shape
+        rp = _rows_pad(q_len)
+        o_part = torch.zeros((batch, heads, rp, d), dtype=torch.float32, device=q.device)
+        lse = torch.full((batch, heads, rp), -math.inf, dtype=torch.float32, device=q.device)
+    og, lg = _gather(o_part, group), _gather(lse, group)
+    ranks = [r for r in range(world) if shard_valid(kv_len, world, r) > 0]
+    if len(ranks) < world:
+        og, lg = og[ranks].contiguous(), lg[ranks].contiguous()
+    return backend.combine(og, lg, q.shape[1])

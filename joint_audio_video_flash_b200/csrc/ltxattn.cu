@@ -56,6 +56,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_check",         "ltxattn_destroy",          "ltxattn_status_string",
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
     "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope", "ltxattn_na3d_forward",
+    "ltxattn_forward_partial", "ltxattn_combine",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -700,6 +701,95 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
         : best == 1 ? launch_na<128, 1, 8, 16>(tq, tk, tv, to, p, c->num_sms, stream)
                     : launch_na<128, 4, 4, 8>(tq, tk, tv, to, p, c->num_sms, stream);
   }
+  return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
+int ltxattn_forward_partial(const void* q, const void* k, const void* v, float* o_part,
+                            float* lse, int q_len, int kv_len, int kv_valid_len, int batch,
+                            int heads, int head_dim, float scale, ltxattn_stream_t stream_) {
+  if (!o_part || !lse) return LTXATTN_ERR_INVALID_ARG;
+  // q, k, v and a stand-in for the bf16 output: the same checks as ltxattn_forward
+  int st = validate(q, k, v, o_part, q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale);
+  if (st != LTXATTN_OK) return st;
+  if (reinterpret_cast<uintptr_t>(lse) & 15u) return LTXATTN_ERR_MISALIGNED;
+  const size_t rows_pad = (size_t)((q_len + ltx::kBlockM - 1) / ltx::kBlockM) * ltx::kBlockM;
+  const size_t n_rows = (size_t)batch * heads * rows_pad;
+  const size_t o_bytes = n_rows * head_dim * 4, l_bytes = n_rows * 4;
+  const size_t row = (size_t)heads * head_dim * 2;
+  const size_t nq = (size_t)batch * q_len * row, nkv = (size_t)batch * kv_len * row;
+  if (overlaps(o_part, o_bytes, q, nq) || overlaps(o_part, o_bytes, k, nkv) ||
+      overlaps(o_part, o_bytes, v, nkv) || overlaps(lse, l_bytes, q, nq) ||
+      overlaps(lse, l_bytes, k, nkv) || overlaps(lse, l_bytes, v, nkv) ||
+      overlaps(lse, l_bytes, o_part, o_bytes))
+    return LTXATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  Context* c = current_context(&st);
+  if (!c) return st;
+
+  FwdParams p{};
+  p.q_len = q_len;
+  p.kv_len = kv_len;
+  p.kv_valid = kv_valid_len;
+  p.heads = heads;
+  p.batch = batch;
+  p.n_q_tiles = (q_len + ltx::kBlockM - 1) / ltx::kBlockM;
+  p.n_kv_tiles = (kv_valid_len + ltx::kBlockN - 1) / ltx::kBlockN;
+  p.num_splits = 1;
+  p.tiles_per_split = p.n_kv_tiles;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = c->d_status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  p.o_part = o_part;
+  p.lse_part = lse;
+  // the output map is never stored through in split mode; q's map stands in for it
+  CUtensorMap tq, tk, tv;
+  if (!encode_bshd(*c, &tq, q, q_len, batch, heads, head_dim) ||
+      !encode_bshd(*c, &tk, k, kv_len, batch, heads, head_dim) ||
+      !encode_bshd(*c, &tv, v, kv_len, batch, heads, head_dim))
+    return LTXATTN_ERR_CUDA;
+  const bool dual = head_dim == 64 && p.n_kv_tiles > ltx::kSkvMaxKvTiles &&
+                    p.n_q_tiles <= kDualMaxQTiles;
+  cudaError_t e;
+  if (dual)
+    e = launch_fwd<64, true, 1>(tq, tk, tv, tq, p, stream);
+  else if (head_dim == 64)
+    e = launch_attention<64, true>(tq, tk, tv, tq, p, stream);
+  else
+    e = launch_attention<128, true>(tq, tk, tv, tq, p, stream);
+  return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
+int ltxattn_combine(const float* o_parts, const float* lses, void* out, int parts, int q_len,
+                    int batch, int heads, int head_dim, ltxattn_stream_t stream_) {
+  if (!o_parts || !lses || !out) return LTXATTN_ERR_INVALID_ARG;
+  if (parts < 1 || q_len < 1 || batch < 1 || heads < 1) return LTXATTN_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LTXATTN_ERR_UNSUPPORTED;
+  if (q_len > LTXATTN_MAX_LEN || heads > LTXATTN_MAX_HEADS || batch > LTXATTN_MAX_BATCH ||
+      parts > 65536)
+    return LTXATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(o_parts) | reinterpret_cast<uintptr_t>(lses) |
+       reinterpret_cast<uintptr_t>(out)) & 15u)
+    return LTXATTN_ERR_MISALIGNED;
+  FwdParams p{};
+  p.q_len = q_len;
+  p.heads = heads;
+  p.batch = batch;
+  p.n_q_tiles = (q_len + ltx::kBlockM - 1) / ltx::kBlockM;
+  p.num_splits = parts;
+  const size_t n_rows = (size_t)parts * batch * heads * p.n_q_tiles * ltx::kBlockM;
+  const size_t out_bytes = (size_t)batch * q_len * heads * head_dim * 2;
+  if (overlaps(out, out_bytes, o_parts, n_rows * head_dim * 4) ||
+      overlaps(out, out_bytes, lses, n_rows * 4))
+    return LTXATTN_ERR_INVALID_ARG;
+  const long long blocks =
+      ((long long)batch * q_len * heads * (head_dim / 4) + ltx::kCombineThreads - 1) /
+      ltx::kCombineThreads;
+  if (blocks > 0x7fffffffLL) return LTXATTN_ERR_UNSUPPORTED;
+  p.o_part = const_cast<float*>(o_parts);
+  p.lse_part = const_cast<float*>(lses);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const cudaError_t e = head_dim == 64 ? launch_combine<64>(p, out, stream)
+                                       : launch_combine<128>(p, out, stream);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 

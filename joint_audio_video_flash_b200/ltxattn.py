@@ -52,6 +52,8 @@ def load() -> ctypes.CDLL:
             lib.ltxattn_qk_norm_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                                  cf, vp]
             lib.ltxattn_na3d_forward.argtypes = [vp, vp, vp, vp] + [ci] * 9 + [cf, vp]
+            lib.ltxattn_forward_partial.argtypes = [vp, vp, vp, vp, vp] + [ci] * 6 + [cf, vp]
+            lib.ltxattn_combine.argtypes = [vp, vp, vp] + [ci] * 5 + [vp]
             lib.ltxattn_entry_point_name.argtypes = [ci]
             lib.ltxattn_entry_point_name.restype = ctypes.c_char_p
             _lib = lib
@@ -230,4 +232,74 @@ def na3d_forward(q, k, v, grid, window, out=None, *, scale: float | None = None,
         grid_y, grid_x, int(heads), int(head_dim), win_t, win_y, win_x, ctypes.c_float(scale),
         ctypes.c_void_p(_stream_handle(stream)))
     _check(st, "ltxattn_na3d_forward")
+    return out
+
+
+def rows_pad(q_len: int) -> int:
+    """Query rows per (batch, head) in the partial-result layout: q_len rounded up to 128."""
+    return -(-int(q_len) // 128) * 128
+
+
+def forward_partial(q, k, v, o_part=None, lse=None, *, kv_valid_len: int | None = None,
+                    scale: float | None = None, stream=None):
+    """Attention over one key range (``ltxattn_forward_partial``): returns (o_part, lse).
+
+    q: [B, Lq, H, D]; k, v: [B, Lkv, H, D] (bf16 CUDA).  o_part: fp32 [B, H, rows_pad, D],
+    lse: fp32 [B, H, rows_pad] base-2 log-sum-exp; rows past Lq are left unwritten.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [batch, len, heads, head_dim] tensor")
+    batch, q_len, heads, head_dim = q.shape
+    kv_len = k.shape[1]
+    if tuple(k.shape) != (batch, kv_len, heads, head_dim) or v.shape != k.shape:
+        raise ValueError("k and v must be [batch, kv_len, heads, head_dim] matching q")
+    rp = rows_pad(q_len)
+    if o_part is None:
+        o_part = torch.empty(batch, heads, rp, head_dim, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(batch, heads, rp, dtype=torch.float32, device=q.device)
+    if (o_part.dtype != torch.float32 or tuple(o_part.shape) != (batch, heads, rp, head_dim)
+            or not o_part.is_contiguous() or lse.dtype != torch.float32
+            or tuple(lse.shape) != (batch, heads, rp) or not lse.is_contiguous()):
+        raise ValueError("o_part / lse must be contiguous fp32 [B, H, rows_pad, D] / [B, H, rows_pad]")
+    if kv_valid_len is None:
+        kv_valid_len = kv_len
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    st = load().ltxattn_forward_partial(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o_part.data_ptr()),
+        ctypes.c_void_p(lse.data_ptr()), int(q_len), int(kv_len), int(kv_valid_len), int(batch),
+        int(heads), int(head_dim), ctypes.c_float(scale), ctypes.c_void_p(_stream_handle(stream)))
+    _check(st, "ltxattn_forward_partial")
+    return o_part, lse
+
+
+def combine(o_parts, lses, q_len: int, out=None, *, stream=None):
+    """Merge of key-range partial results (``ltxattn_combine``) into bf16 [B, q_len, H, D].
+
+    o_parts: fp32 [P, B, H, rows_pad, D]; lses: fp32 [P, B, H, rows_pad].
+    """
+    import torch
+    if (not isinstance(o_parts, torch.Tensor) or o_parts.dtype != torch.float32
+            or o_parts.dim() != 5 or not o_parts.is_contiguous() or not o_parts.is_cuda):
+        raise TypeError("o_parts must be a contiguous fp32 CUDA [P, B, H, rows_pad, D] tensor")
+    parts, batch, heads, rp, head_dim = o_parts.shape
+    if rp != rows_pad(q_len):
+        raise ValueError(f"rows_pad {rp} does not match q_len {q_len}")
+    if (lses.dtype != torch.float32 or tuple(lses.shape) != (parts, batch, heads, rp)
+            or not lses.is_contiguous()):
+        raise ValueError("lses must be a contiguous fp32 [P, B, H, rows_pad] tensor")
+    if out is None:
+        out = torch.empty(batch, q_len, heads, head_dim, dtype=torch.bfloat16,
+                          device=o_parts.device)
+    st = load().ltxattn_combine(
+        ctypes.c_void_p(o_parts.data_ptr()), ctypes.c_void_p(lses.data_ptr()),
+        ctypes.c_void_p(out.data_ptr()), int(parts), int(q_len), int(batch), int(heads),
+        int(head_dim), ctypes.c_void_p(_stream_handle(stream)))
+    _check(st, "ltxattn_combine")
     return out

@@ -142,6 +142,44 @@ def test_qk_norm_rope_host_validation(lib, kw, status):
     assert qk(lib, **kw) == status
 
 
+def partial(lib, q=Q, k=K, v=V, o=O, lse=O + (1 << 24), q_len=128, kv_len=128, valid=128,
+            batch=2, heads=4, d=64, scale=0.125):
+    return lib.ltxattn_forward_partial(*(ctypes.c_void_p(x) for x in (q, k, v, o, lse)),
+                                       q_len, kv_len, valid, batch, heads, d,
+                                       ctypes.c_float(scale), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(lse=0), ltxattn.ERR_INVALID_ARG),
+    (dict(valid=0), ltxattn.ERR_INVALID_ARG),
+    (dict(d=96), ltxattn.ERR_UNSUPPORTED),
+    (dict(lse=O + (1 << 24) + 4), ltxattn.ERR_MISALIGNED),
+    (dict(o=K), ltxattn.ERR_INVALID_ARG),                  # o_part overlaps k
+    (dict(lse=Q + 1024), ltxattn.ERR_INVALID_ARG),         # lse overlaps q
+    (dict(lse=O + 4096), ltxattn.ERR_INVALID_ARG),         # lse overlaps o_part
+])
+def test_forward_partial_host_validation(lib, kw, status):
+    assert partial(lib, **kw) == status
+
+
+def comb(lib, o=O, lse=O + (1 << 24), out=Q, parts=2, q_len=100, batch=2, heads=4, d=64):
+    return lib.ltxattn_combine(ctypes.c_void_p(o), ctypes.c_void_p(lse), ctypes.c_void_p(out),
+                               parts, q_len, batch, heads, d, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(out=0), ltxattn.ERR_INVALID_ARG),
+    (dict(parts=0), ltxattn.ERR_INVALID_ARG),
+    (dict(q_len=0), ltxattn.ERR_INVALID_ARG),
+    (dict(d=32), ltxattn.ERR_UNSUPPORTED),
+    (dict(parts=65537), ltxattn.ERR_UNSUPPORTED),
+    (dict(out=Q + 8), ltxattn.ERR_MISALIGNED),
+    (dict(out=O + 1024), ltxattn.ERR_INVALID_ARG),         # out overlaps the partials
+])
+def test_combine_host_validation(lib, kw, status):
+    assert comb(lib, **kw) == status
+
+
 def test_new_calls_reach_cuda_with_valid_arguments(lib):
     import torch
     if torch.cuda.is_available():
@@ -149,3 +187,5 @@ def test_new_calls_reach_cuda_with_valid_arguments(lib):
     assert na3d(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
     assert qk(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
     assert qk(lib, qo=Q, ko=K) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)  # in place
+    assert partial(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
+    assert comb(lib) == ltxattn.ERR_CUDA
