@@ -8,8 +8,8 @@ by default", Description).  Two exchange patterns cover the block's attentions:
 
 * self-attention over a sharded sequence (video self): every rank gathers all shards of K
   and V, computes its own queries' attention over each shard as a partial result (fp32
-  output and base-2 log-sum-exp, ``ltxattn_forward_partial``) and merges the partials
-  (``ltxattn_combine``);
+  output and base-2 log-sum-exp, ``ltxattn_forward_partial``; its own shard first, while
+  the gathers run) and merges the partials (``ltxattn_combine``);
 * replicated queries over sharded keys and values (v2a: audio queries, video keys): every
   rank computes the partial over its own shard; the partials and their statistics are
   all-gathered and merged, so every rank ends with the full result.
@@ -52,14 +52,15 @@ def shard_valid(total: int, world: int, rank: int) -> int:
     return max(0, min(ls, int(total) - rank * ls))
 
 
-def _gather(t, group):
-    """[world, *t.shape] stack of every rank's t (rank order)."""
+def _gather(t, group, async_op: bool = False):
+    """[world, *t.shape] stack of every rank's t (rank order); with async_op, also the
+    collective's handle (wait on it before reading other ranks' slices)."""
     import torch
     import torch.distributed as dist
     world = dist.get_world_size(group)
     out = torch.empty((world, *t.shape), dtype=t.dtype, device=t.device)
-    dist.all_gather(list(out.unbind(0)), t.contiguous(), group=group)
-    return out
+    work = dist.all_gather(list(out.unbind(0)), t.contiguous(), group=group, async_op=async_op)
+    return (out, work) if async_op else out
 
 
 def _rows_pad(q_len: int) -> int:
@@ -83,16 +84,25 @@ def self_attention(q_local, k_local, v_local, seq_len: int, group, *, scale: flo
             v_local.shape != q_local.shape:
         raise ValueError(f"shards must be [B, {shard_len(seq_len, world)}, H, D] on every rank")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    kb, vb = _gather(k_local, group), _gather(v_local, group)
+    rank = dist.get_rank(group)
+    # the gathers run while this rank's own shard, already local, gives its partial
+    (kb, wk), (vb, wv) = _gather(k_local, group, True), _gather(v_local, group, True)
     ranks = [r for r in range(world) if shard_valid(seq_len, world, r) > 0]
     rp = _rows_pad(ls)
     o_parts = torch.empty((len(ranks), batch, heads, rp, d), dtype=torch.float32,
                           device=q_local.device)
     lses = torch.empty((len(ranks), batch, heads, rp), dtype=torch.float32,
                        device=q_local.device)
-    for i, r in enumerate(ranks):
-        backend.partial(q_local, kb[r], vb[r], shard_valid(seq_len, world, r), scale,
+    if rank in ranks:
+        i = ranks.index(rank)
+        backend.partial(q_local, k_local, v_local, shard_valid(seq_len, world, rank), scale,
                         o_parts[i], lses[i])
+    wk.wait()
+    wv.wait()
+    for i, r in enumerate(ranks):
+        if r != rank:
+            backend.partial(q_local, kb[r], vb[r], shard_valid(seq_len, world, r), scale,
+                            o_parts[i], lses[i])
     return backend.combine(o_parts, lses, ls)
 
 
