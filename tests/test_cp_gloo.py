@@ -112,6 +112,52 @@ def test_two_ranks_match_whole_sequence_attention():
             assert err <= 2e-2, (rank, name, err)
 
 
+def _run_tiny(rank, world, port, q):
+    # 5 tokens over 4 ranks: shards of 2, 2, 1 and 0 real tokens
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    from joint_audio_video_flash_b200 import cp, synth
+    from oracle import oracle
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    be = OracleBackend()
+    n, h, d = 5, 1, 64
+    qg, kg, vg = synth.make_qkv(1, n, n, h, d, seed=903)
+    ls = cp.shard_len(n, world)
+    lo, hi = min(n, rank * ls), min(n, (rank + 1) * ls)
+    pad = lambda t: torch.nn.functional.pad(t[:, lo:hi], (0, 0, 0, 0, 0, ls - (hi - lo)))  # noqa: E731
+    out = cp.self_attention(pad(qg), pad(kg), pad(vg), n, dist.group.WORLD, backend=be)
+    ref = oracle.attention(qg, kg, vg, d ** -0.5)[:, lo:hi]
+    err_self = float(np.abs(out[:, : hi - lo].double().numpy() - ref).max()) if hi > lo else 0.0
+    qa, _, _ = synth.make_qkv(1, 3, 3, h, d, seed=904)
+    out2 = cp.cross_attention(qa, pad(kg), pad(vg), n, dist.group.WORLD, backend=be)
+    err_cross = float(np.abs(out2.double().numpy() - oracle.attention(qa, kg, vg, d ** -0.5)).max())
+    q.put((rank, {"self": err_self, "cross": err_cross}))
+    dist.destroy_process_group()
+
+
+def test_four_ranks_with_an_empty_shard():
+    world, port = 4, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_run_tiny, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=240) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert len(results) == world
+    for rank, res in results.items():
+        for name, err in res.items():
+            assert err <= 2e-2, (rank, name, err)
+
+
 def test_shard_bounds():
     from joint_audio_video_flash_b200 import cp
     assert cp.shard_len(300, 2) == 150 and cp.shard_len(257, 2) == 129
