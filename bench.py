@@ -38,11 +38,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, keyed by
 # the hash of the sources that make up that kernel; reported as null once they change.
 KERNEL_SOURCES = {
-    "video_self": ("joint_audio_video_flash_b200/csrc/fmha_fwd_pp.cuh",
-                   "joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
+    "video_self": ("joint_audio_video_flash_b200/csrc/attn_fwd_pp.cuh",
+                   "joint_audio_video_flash_b200/csrc/attn_fwd.cuh",
                    "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
     "na3d_decoder": ("joint_audio_video_flash_b200/csrc/na3d_fwd.cuh",
-                     "joint_audio_video_flash_b200/csrc/fmha_fwd.cuh",
+                     "joint_audio_video_flash_b200/csrc/attn_fwd.cuh",
                      "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
     "qk_prologue": ("joint_audio_video_flash_b200/csrc/qk_prologue.cuh",
                     "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
@@ -62,12 +62,12 @@ def kernel_label(c, num_sms: int = 148) -> str:
     qt = -(-c.q_len // 128)
     kt = -(-c.kv_valid_len // 128)
     if kt <= 2 and c.batch * c.heads * qt > num_sms:
-        return f"fmha_fwd_skv_sm100<{kt}> (persistent, K/V resident)"
+        return f"ltx_attn_fwd_skv<{kt}> (persistent, K/V resident)"
     if c.head_dim == 64 and kt > 2 and qt <= 1:
-        return "fmha_fwd_sm100<64, 1 S buffer> (two CTAs per SM)"
+        return "ltx_attn_fwd<64, 1 S buffer> (two CTAs per SM)"
     if qt >= 2:
-        return f"fmha_fwd_pp_sm100<{c.head_dim}> (two 128-row query tiles per CTA)"
-    return f"fmha_fwd_sm100<{c.head_dim}>"
+        return f"ltx_attn_fwd_pp<{c.head_dim}> (two 128-row query tiles per CTA)"
+    return f"ltx_attn_fwd<{c.head_dim}>"
 
 
 def kernel_source_hash(kernel: str = "video_self") -> str:
@@ -160,6 +160,91 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+class NvmlClockTrace:
+    """The SM clock read through NVML (read-only queries) every `period_s` on a host thread,
+    each reading stamped with the host wall clock, so that per-call device times can be put
+    beside the clock they ran at (nvidia-smi's 200 ms samples are coarser than one call)."""
+
+    def __init__(self, uuid: str | None, period_s: float = 0.002):
+        self.uuid, self.period_s = uuid, period_s
+        self.samples = []  # (wall time s, SM MHz)
+        self._stop = None
+        self._thread = None
+        self.max_mhz = None
+
+    def __enter__(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                except Exception:
+                    break
+                self.samples.append((time.time(), float(mhz)))
+                self._stop.wait(self.period_s)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+
+    def mhz_during(self, t0: float, t1: float):
+        """Mean SM MHz of the readings in [t0, t1], else the reading nearest to the middle."""
+        if not self.samples:
+            return None
+        inside = [m for t, m in self.samples if t0 <= t <= t1]
+        if inside:
+            return sum(inside) / len(inside)
+        mid = 0.5 * (t0 + t1)
+        return min(self.samples, key=lambda tm: abs(tm[0] - mid))[1]
+
+
+def clock_normalised(us, wall, trace):
+    """Per-call times at the maximum SM clock: t x (MHz the call ran at / max MHz), with the
+    calls binned by clock.  `us` and `wall` ([start, end] host seconds) are per call."""
+    if trace is None or not trace.samples or not trace.max_mhz:
+        return None
+    mhz = [trace.mhz_during(a, b) for a, b in wall]
+    norm = [t * f / trace.max_mhz for t, f in zip(us, mhz)]
+    bins = {}
+    for t, f in zip(us, mhz):
+        lo = int(f // 100) * 100
+        bins.setdefault(lo, []).append(t)
+    return {"us_median_at_max_clock": statistics.median(norm),
+            "us_p10_at_max_clock": pct(norm, 0.1), "us_p90_at_max_clock": pct(norm, 0.9),
+            "mhz_median": statistics.median(mhz), "mhz_min": min(mhz), "mhz_max_seen": max(mhz),
+            "sm_max_mhz": trace.max_mhz, "nvml_samples": len(trace.samples),
+            "by_clock": [{"mhz": [lo, lo + 100], "calls": len(v), "us_median": statistics.median(v)}
+                         for lo, v in sorted(bins.items())]}
+
+
+def pct(xs, f):
+    s = sorted(xs)
+    return s[min(len(s) - 1, max(0, int(f * len(s))))]
+
+
+def device_uuid(dev):
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+
+
 # --------------------------------------------------------------------------- oracle sample
 def oracle_sample(calls, fraction: float, seed: int):
     """Time the fp64 oracle on ``fraction`` of every call's query rows (same mix of work)."""
@@ -205,6 +290,221 @@ def cpu_baseline(calls, target_s: float, seed: int = 0):
             "kind": "oracle",
             "sample": f"{rows} query rows ({frac:.4%} of every call's real rows, same work mix), "
                       f"{fl:.3e} FLOP in {s:.1f} s, fp64, OpenMP over rows"}
+
+
+# --------------------------------------------------------------------------- per-config table
+# Every workload of the attention set (the block768 set is the headline line itself) and the
+# next rows' workloads, each timed on its own, with parity against the oracle on sampled rows
+# computed after its timed loop.
+PER_CONFIG_ATTENTION = ("tiny", "video15360_b1", "audio_stream", "longclip", "text_xattn")
+L2_FLUSH_BYTES = 256 << 20  # written before every timed call: L2 (126 MB) holds no input
+
+
+def parity_stats(got, ref):
+    """max-abs, relative L2 and cosine of a GPU result against the fp64 oracle."""
+    import numpy as np
+    g = np.asarray(got, dtype=np.float64).reshape(ref.shape)
+    d = g - ref
+    nr = float(np.linalg.norm(ref))
+    return {"max_abs": float(np.abs(d).max()),
+            "rel_l2": float(np.linalg.norm(d) / nr) if nr else None,
+            "cos": float((g * ref).sum() / (np.linalg.norm(g) * nr)) if nr else None,
+            "finite": bool(np.all(np.isfinite(g)))}
+
+
+def attention_parity(c, q, k, v, out_dev, seed):
+    """The oracle on every row of a small call, else on sampled rows: 2 seeded rows of every
+    (batch, head) and the last 16 real rows of the last head (the ragged tail)."""
+    import torch
+
+    from joint_audio_video_flash_b200 import synth
+    from oracle import oracle
+    n_rows = c.batch * c.q_len * c.heads
+    rows = None
+    if n_rows * c.kv_valid_len > 4e6:
+        r = synth.sample_rows(c.batch, c.q_len, c.heads, 2, seed=seed, full_heads=())
+        i = torch.arange(max(0, c.q_valid - 16), c.q_valid)
+        tail = ((c.batch - 1) * c.q_len + i) * c.heads + (c.heads - 1)
+        rows = torch.unique(torch.cat([r, tail]))
+    ref = oracle.attention(q, k, v, c.scale, kv_valid_len=c.kv_valid_len,
+                           rows=None if rows is None else rows.numpy())
+    got = out_dev.cpu().to(torch.float64)
+    got = got.numpy() if rows is None else got.reshape(-1, c.head_dim)[rows].numpy()
+    st = parity_stats(got, ref)
+    st["rows"] = int(n_rows if rows is None else len(rows))
+    return st
+
+
+def call_roofline(flops, nbytes, us, peaks):
+    """TFLOP/s, GB/s and the fraction of the binding measured peak (by arithmetic intensity
+    against the ridge of the measured bf16 burst peak and HBM bandwidth)."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tfl = flops / (us * 1e-6) / 1e12
+    gbs = nbytes / (us * 1e-6) / 1e9
+    tensor = flops / nbytes > burst * 1e12 / (hbm * 1e9)
+    return {"tflops": tfl, "frac_bf16_peak": tfl / burst, "gbs": gbs, "frac_hbm": gbs / hbm,
+            "bound": "tensor" if tensor else "hbm",
+            "frac_of_bound": tfl / burst if tensor else gbs / hbm}
+
+
+def timed_calls(fns, steps, warmup, stream, flush):
+    """Runs every fn of `fns` once per step, each bracketed by CUDA events on `stream` after an
+    L2 flush (outside the events); returns per-fn lists of µs and of host-wall intervals."""
+    import torch
+    for _ in range(warmup):
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in fns] for _ in range(steps)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    e0.record(stream)
+    for s in range(steps):
+        for i, f in enumerate(fns):
+            if flush is not None:
+                flush.zero_()
+            ev[s][i][0].record(stream)
+            f()
+            ev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    us = [[ev[s][i][0].elapsed_time(ev[s][i][1]) * 1e3 for s in range(steps)]
+          for i in range(len(fns))]
+    wall = [[(wall0 + e0.elapsed_time(ev[s][i][0]) * 1e-3, wall0 + e0.elapsed_time(ev[s][i][1]) * 1e-3)
+             for s in range(steps)] for i in range(len(fns))]
+    return us, wall
+
+
+def dist_stats(us):
+    return {"us_median": statistics.median(us), "us_p10": pct(us, 0.1), "us_p90": pct(us, 0.9)}
+
+
+def measure_attention_config(name, steps, warmup, peaks, dev, stream, flush, trace):
+    import torch
+
+    from joint_audio_video_flash_b200 import ltxattn, synth, workloads
+    desc, calls = workloads.configs()[name]
+    host, ins, outs = [], [], []
+    for c in calls:
+        trip = synth.make_qkv(c.batch, c.q_len, c.kv_len, c.heads, c.head_dim, c.seed,
+                              q_valid=c.q_valid, kv_valid=c.kv_valid_len)
+        host.append(trip)
+        ins.append(tuple(t.to(dev) for t in trip))
+        outs.append(torch.empty_like(ins[-1][0]))
+
+    def fn(i):
+        c = calls[i]
+        return lambda: ltxattn.forward(*ins[i], outs[i], kv_valid_len=c.kv_valid_len,
+                                       scale=c.scale)
+
+    us, wall = timed_calls([fn(i) for i in range(len(calls))], steps, warmup, stream, flush)
+    ltxattn.check()
+    out = {"description": desc, "steps": steps, "l2": "flushed before every call", "calls": {}}
+    tot_us = 0.0
+    for i, c in enumerate(calls):
+        d = dist_stats(us[i])
+        d.update(call_roofline(c.flops, c.bytes, d["us_median"], peaks))
+        d["shape"] = (f"B{c.batch} Lq{c.q_len} Lkv{c.kv_len} valid{c.kv_valid_len} "
+                      f"H{c.heads} D{c.head_dim}")
+        d["kernel"] = kernel_label(c)
+        if c.flops / c.bytes > 1000:  # tensor-bound calls: the clock decides their time
+            d["clock"] = clock_normalised(us[i], wall[i], trace)
+        d["parity"] = attention_parity(c, *host[i], outs[i], seed=c.seed)
+        out["calls"][c.name] = d
+        tot_us += d["us_median"]
+    flops = sum(c.flops for c in calls)
+    out.update({"us_sum_of_medians": tot_us, "tflops": flops / (tot_us * 1e-6) / 1e12})
+    del ins, outs
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_prologue_config(steps, warmup, peaks, dev, stream):
+    import torch
+
+    from joint_audio_video_flash_b200 import ltxattn, synth
+    from oracle import qk_prologue as qp
+    b, l, h, d = PROLOGUE_SHAPE
+    host = synth.make_qk_prologue_inputs(b, l, h, d, seed=PROLOGUE_SEED)
+    dq, dk, dwq, dwk, dcos, dsin = (t.to(dev) for t in host)
+    qo, ko = torch.empty_like(dq), torch.empty_like(dk)
+    us, _ = timed_calls([lambda: ltxattn.qk_norm_rope(dq, dk, dwq, dwk, dcos, dsin, qo, ko)],
+                        steps, warmup, stream, None)
+    nbytes = prologue_step_bytes()
+    r = dist_stats(us[0])
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    r.update({"gbs": nbytes / (r["us_median"] * 1e-6) / 1e9, "bound": "hbm",
+              "l2": "inputs larger than L2", "steps": steps,
+              "kernel": "ltx_qk_norm_rope<4, 4, 2>", "description": prologue_config(1)["description"]})
+    r["frac_hbm"] = r["gbs"] / hbm
+    # parity: the first 256 and the last 64 tokens of every batch element, q and k
+    q, k, wq, wk, cos, sin = host
+    worst = None
+    for sl in (slice(0, 256), slice(l - 64, l)):
+        for x, w, o in ((q, wq, qo), (k, wk, ko)):
+            st = parity_stats(o[:, sl].cpu().to(torch.float64).numpy(),
+                              qp.rms_norm_rope(x[:, sl], w, cos[sl], sin[sl], 1e-6))
+            if worst is None or st["rel_l2"] > worst["rel_l2"]:
+                worst = st
+    worst["rows"] = "tokens 0..255 and the last 64 of both batch elements, q and k (worst part)"
+    r["parity"] = worst
+    del dq, dk, qo, ko
+    torch.cuda.empty_cache()
+    return r
+
+
+def measure_na3d_config(steps, warmup, peaks, dev, stream):
+    import numpy as np
+    import torch
+
+    from joint_audio_video_flash_b200 import ltxattn, synth
+    from oracle import na3d as na
+    grid, window, heads, d, b = NA_GRID, NA_WINDOW, NA_HEADS, NA_D, NA_BATCH
+    n = grid[0] * grid[1] * grid[2]
+    q, k, v = synth.make_qkv(b, n, n, heads, d, seed=NA_SEED)
+    dq, dk, dv = (t.to(dev) for t in (q, k, v))
+    out = torch.empty_like(dq)
+    us, _ = timed_calls([lambda: ltxattn.na3d_forward(dq, dk, dv, grid, window, out)],
+                        steps, warmup, stream, None)
+    ltxattn.check()
+    r = dist_stats(us[0])
+    flops = na3d_step_flops()
+    issued = na_key_tiles(grid, window) * b * heads * 4.0 * 128 * 128 * d
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tfl = flops / (r["us_median"] * 1e-6) / 1e12
+    r.update({"tflops": tfl, "frac_bf16_peak": tfl / burst, "bound": "tensor",
+              "issued_tflops": issued / (r["us_median"] * 1e-6) / 1e12, "density": flops / issued,
+              "l2": "inputs larger than L2", "steps": steps,
+              "description": na3d_config(1)["description"]})
+    # parity on 192 tokens: the grid's corners and edges and seeded interior tokens
+    g = np.random.default_rng(NA_SEED)
+    rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(n - 64, n),
+                                     g.integers(0, n, 64)]))
+    ref = na.na3d(q, k, v, grid, window, d ** -0.5, rows=rows)
+    got = out.cpu().to(torch.float64)[:, torch.as_tensor(rows)].numpy()
+    r["parity"] = parity_stats(got, ref)
+    r["parity"]["rows"] = f"{len(rows)} tokens x {heads} heads"
+    del dq, dk, dv, out
+    torch.cuda.empty_cache()
+    return r
+
+
+def per_config_table(args, peaks, dev, stream):
+    import torch
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    table = {}
+    with NvmlClockTrace(device_uuid(dev)) as trace:
+        for name in PER_CONFIG_ATTENTION:
+            table[name] = measure_attention_config(name, args.per_config_steps, 3, peaks, dev,
+                                                   stream, flush, trace)
+        table["qk_prologue"] = measure_prologue_config(args.per_config_steps, 3, peaks, dev,
+                                                       stream)
+        table["na3d_decoder"] = measure_na3d_config(args.per_config_steps, 3, peaks, dev, stream)
+    del flush
+    torch.cuda.empty_cache()
+    return table
 
 
 # --------------------------------------------------------------------------- dist
@@ -349,9 +649,10 @@ def run_ltxattn(args):
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         uuid = None
-    with ClockSampler(uuid) as clocks:
+    with ClockSampler(uuid) as clocks, NvmlClockTrace(uuid) as trace:
         barrier(world)
         torch.cuda.synchronize()
+        wall0 = time.time()
         t_start.record(stream)
         for s in range(args.steps):
             step(per_call[s])
@@ -365,10 +666,13 @@ def run_ltxattn(args):
     step_flops = sum(c.flops for c in calls)
     value = whole_job_tflops(step_flops, args.steps, world, total_ms)
 
-    call_us = []
+    call_us, call_wall = [], []
     for i, c in enumerate(calls):
         ts = [per_call[s][i][0].elapsed_time(per_call[s][i][1]) * 1e3 for s in range(args.steps)]
         call_us.append(ts)
+        call_wall.append([(wall0 + t_start.elapsed_time(per_call[s][i][0]) * 1e-3,
+                           wall0 + t_start.elapsed_time(per_call[s][i][1]) * 1e-3)
+                          for s in range(args.steps)])
     launches_per_step = sum(1 if sp == 1 else 2 for sp in splits)
 
     # ---- end to end through the public API with host buffers.  Every step uploads all
@@ -480,6 +784,10 @@ def run_ltxattn(args):
             "shape": f"B{c.batch} Lq{c.q_len} Lkv{c.kv_len} valid{c.kv_valid_len} "
                      f"H{c.heads} D{c.head_dim}",
             "splits": splits[i], "kernel": kernel_label(c)}
+        if c.flops / c.bytes > 1000:  # tensor-bound: time beside the SM clock it ran at
+            per_call_out[c.name]["clock"] = clock_normalised(call_us[i], call_wall[i], trace)
+        if rank == 0 and not args.no_parity:  # the oracle on sampled rows, after the timing
+            per_call_out[c.name]["parity"] = attention_parity(c, *host[i], outs[i], seed=c.seed)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -496,6 +804,10 @@ def run_ltxattn(args):
         "clocks": clk,
         "per_call": per_call_out,
     }
+    if rank == 0 and world == 1 and not args.no_per_config and args.workload == "block768":
+        del dev_in, pinned
+        torch.cuda.empty_cache()
+        line["per_config"] = per_config_table(args, peaks, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(calls, args.cpu_seconds)
     if rank == 0:
@@ -725,7 +1037,7 @@ def run_prologue(args):
         "config": prologue_config(world),
         "roofline": {"bound": "hbm", "achieved": value, "peak": hbm, "unit": "GB/s",
                      "frac": value / hbm, "traffic": traffic_per_launch("qk_prologue"),
-                     "kernel": "qk_norm_rope<4, 4, 2>",
+                     "kernel": "ltx_qk_norm_rope<4, 4, 2>",
                      "algorithmic_bytes": step_bytes, "peak_source": f"{peak_src} hbm_gbs"},
         "e2e": {"value": step_bytes * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": 2 * q.numel() * 2, "d2h_bytes_per_step": 2 * q.numel() * 2},
@@ -847,7 +1159,7 @@ def run_na3d(args):
         "config": na3d_config(world),
         "roofline": {"bound": "tensor", "achieved": value, "peak": burst, "unit": "TFLOP/s",
                      "frac": value / burst, "traffic": traffic_per_launch("na3d_decoder"),
-                     "kernel": "na3d_fwd_sm100<128, 2, 8, 8>",
+                     "kernel": "ltx_na3d_fwd<128, 2, 8, 8>",
                      "issued_tflops": issued_tflops, "issued_frac": issued_tflops / burst,
                      "density": step_flops / issued,
                      "peak_source": f"{peak_src} bf16_tflops (burst)"},
@@ -880,6 +1192,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-config table (every other workload, timed on its own)")
+    ap.add_argument("--no-parity", action="store_true",
+                    help="skip the oracle comparison of the timed outputs")
+    ap.add_argument("--per-config-steps", type=int, default=10)
     ap.add_argument("--once", action="store_true",
                     help="run each call of the workload once and exit (profiling)")
     args = ap.parse_args()

@@ -31,7 +31,10 @@
  *
  * Threading.  Calls on one device may come from any host thread.  Calls on the
  * same stream are ordered by the stream; calls on different streams use separate
- * workspaces.
+ * workspaces.  A call that needs the key-split workspace holds a per-device lock from
+ * the workspace lookup (and any grow) through its launches, so host threads sharing a
+ * stream never launch on a buffer another thread is replacing.  ltxattn_destroy must
+ * not run concurrently with other calls on the same device.
  *
  * Errors.  Every entry point returns an ltxattn_status.  Argument checks run on
  * the host, before any CUDA call and before anything is enqueued, so a rejected
@@ -119,9 +122,13 @@ LTXATTN_API int ltxattn_forward_ex(const void* q, const void* k, const void* v, 
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
- * current device.  Returns LTXATTN_ERR_DEVICE_TIMEOUT if a kernel recorded a
- * stalled wait since the last check, LTXATTN_ERR_CUDA if the synchronisation
- * failed, LTXATTN_ERR_NOT_INITIALIZED without a context, else LTXATTN_OK.
+ * current device: the context's word (ltxattn_create) and, if
+ * ltxattn_forward_split_noalloc was ever called on this device, that call's own
+ * word in its scratch array (read with a plain device-to-host copy; nothing is
+ * allocated).  Returns LTXATTN_ERR_DEVICE_TIMEOUT if a kernel recorded a stalled
+ * wait since the last check, LTXATTN_ERR_CUDA if the synchronisation or a copy
+ * failed, LTXATTN_ERR_NOT_INITIALIZED when neither word exists on this device,
+ * else LTXATTN_OK.
  */
 LTXATTN_API int ltxattn_check(ltxattn_stream_t stream);
 
@@ -258,17 +265,20 @@ LTXATTN_API int ltxattn_combine(const float* o_parts, const float* lses, void* o
  * workspace (and ltxattn_create allocates the status word); this call never does.
  * It needs no ltxattn_create.
  *
- * It computes exactly what ltxattn_forward computes, always through the key-range
- * split path: per-part fp32 partial outputs and base-2 log-sum-exps, merged by
- * the combine kernel.  Those partials live in one array of
- * LTXATTN_NOALLOC_SCRATCH_BYTES in the library's own device memory (a static
- * device array: every GPU that loads the library holds it until the process
- * exits).  The caller passes inputs and outputs as for ltxattn_forward.
+ * It computes what ltxattn_forward computes, with the same kernels.  When the key
+ * side is split into ranges (v2a-like shapes), the per-part fp32 partial outputs
+ * and base-2 log-sum-exps live in one array of LTXATTN_NOALLOC_SCRATCH_BYTES in
+ * the library's own device memory (a static device array: every GPU that loads
+ * the library holds it until the process exits) and the merge kernel writes
+ * `out`; with one part the attention kernel writes `out` directly and only the
+ * status word of the array is used.  The caller passes inputs and outputs as for
+ * ltxattn_forward.
  *
- *   num_splits  0 = the library's plan, reduced until the partials fit; >= 1 =
- *               that many key-range parts (clamped to the number of 128-key tiles).
- *   Scratch use: 256 + splits * batch * heads * ceil(q_len/128)*128 *
- *               (head_dim + 1) * 4 bytes must not exceed
+ *   num_splits  0 = the library's plan, capped at the most parts whose partials
+ *               fit (one part always fits); >= 1 = that many key-range parts
+ *               (clamped to the number of 128-key tiles).
+ *   Scratch use with splits > 1: 256 + splits * batch * heads *
+ *               ceil(q_len/128)*128 * (head_dim + 1) * 4 bytes must not exceed
  *               LTXATTN_NOALLOC_SCRATCH_BYTES, else LTXATTN_ERR_UNSUPPORTED is
  *               returned and nothing is enqueued.
  *
@@ -281,7 +291,9 @@ LTXATTN_API int ltxattn_combine(const float* o_parts, const float* lses, void* o
  * reads is written earlier in the same call.  Calls whose GPU work overlaps (on
  * different streams, or from different host threads without ordering) race on the
  * array and give wrong results: order them.  A kernel wait that runs out is
- * recorded in that status word only; this call does not report it.
+ * recorded in that status word, which each call clears when it starts:
+ * ltxattn_check (which needs no context for this word) reports it, so check after
+ * the call whose result matters and before the next one.
  * Returns LTXATTN_OK once enqueued, or INVALID_ARG / UNSUPPORTED / MISALIGNED (as
  * ltxattn_forward, before any CUDA call), UNSUPPORTED when the scratch is too
  * small, LTXATTN_ERR_CUDA on a failed set-up or launch.

@@ -9,7 +9,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libltxattn.so")
 SOURCES = ["ltxattn.cu"]
-DEPS = ["ltxattn.cu", "fmha_fwd.cuh", "fmha_fwd_pp.cuh", "fmha_fwd_skv.cuh", "qk_prologue.cuh", "na3d_fwd.cuh", "combine.cuh", "sm100_ptx.cuh"]
+DEPS = ["ltxattn.cu", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_fwd_skv.cuh", "qk_prologue.cuh", "na3d_fwd.cuh", "combine.cuh", "sm100_ptx.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared"]
 

@@ -1,4 +1,4 @@
-// fmha_fwd.cuh -- flash-style softmax attention forward for sm_100a.
+// attn_fwd.cuh -- flash-style softmax attention forward for sm_100a.
 //
 // Computes O = softmax(scale * Q K^T + M) V per (batch, head) for the four
 // attentions of an LTX-2 joint audio-video DiT block (video self, audio self,
@@ -167,7 +167,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
 
 template <int D, bool kSplit, int kSBuf = 2>
 __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
-    fmha_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    ltx_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams p) {
   using L = FwdSmem<D, kSBuf>;

@@ -1,9 +1,9 @@
-// fmha_fwd_pp.cuh -- attention forward for long query sides on sm_100a: one CTA owns
+// attn_fwd_pp.cuh -- attention forward for long query sides on sm_100a: one CTA owns
 // TWO 128-row query tiles of the same (batch, head) that share every K/V tile, and
 // two softmax warpgroups ping-pong so the tensor core always has one tile's MMAs to
 // run while the other tile's softmax is computed.
 //
-// Same operation, layout, mask and split mode as fmha_fwd.cuh (video self-attention,
+// Same operation, layout, mask and split mode as attn_fwd.cuh (video self-attention,
 // a2v and the long-key parts of v2a of an LTX-2 block; "LTX-2: replicate audio
 // stream across Ulysses ranks by default", Description).
 //
@@ -22,7 +22,7 @@
 // softmax thread can hold a full 128-score row.
 #pragma once
 
-#include "fmha_fwd.cuh"
+#include "attn_fwd.cuh"
 
 namespace ltx {
 
@@ -77,7 +77,7 @@ __device__ __forceinline__ void reg_alloc_208() {
 
 template <int D, bool kSplit>
 __global__ void __launch_bounds__(kPPThreads, 1)
-    fmha_fwd_pp_sm100(const __grid_constant__ CUtensorMap tm_q,
+    ltx_attn_fwd_pp(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {

@@ -1,9 +1,9 @@
-// fmha_fwd_skv.cuh -- attention forward for a short key side (at most 256 keys) on
+// attn_fwd_skv.cuh -- attention forward for a short key side (at most 256 keys) on
 // sm_100a: a2v (video queries over the padded audio keys/values) of an LTX-2 block
 // ("LTX-2: replicate audio stream across Ulysses ranks by default", Description), at
 // head_dim 64, and the streams' queries over a padded text context at head_dim 64 or
 // 128.  Same operation, layout and key mask as
-// fmha_fwd.cuh.  With every key in one S tile the softmax max is exact, so there is
+// attn_fwd.cuh.  With every key in one S tile the softmax max is exact, so there is
 // no online rescale.  The work is bound by HBM (reading Q, writing O) and by the
 // exponentials, so the design keeps both busy at once:
 //
@@ -27,7 +27,7 @@
 // Registers (setmaxnreg): producer/MMA warpgroup 56, epilogue 104, softmax 176.
 #pragma once
 
-#include "fmha_fwd.cuh"
+#include "attn_fwd.cuh"
 
 namespace ltx {
 
@@ -109,7 +109,7 @@ struct SkvCursor {
 
 template <int D, int NKV>
 __global__ void __launch_bounds__(kSkvThreads, 1)
-    fmha_fwd_skv_sm100(const __grid_constant__ CUtensorMap tm_q,
+    ltx_attn_fwd_skv(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {

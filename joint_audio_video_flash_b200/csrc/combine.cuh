@@ -17,7 +17,7 @@ constexpr int kCombineThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_splits(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+    ltx_attn_combine(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    __nv_bfloat16* __restrict__ out, int num_splits, int batch, int heads, int q_len,
                    int rows_pad) {
   constexpr int kVec = D / 4;

@@ -1,7 +1,7 @@
 // ltxattn.cu -- host side of the C ABI declared in include/ltxattn.h: argument
 // validation, per-device context, TMA tensor maps, key-range split planning,
 // workspace and kernel launches.  No CPU compute path exists: every step of the
-// attention runs in the kernels of fmha_fwd.cuh, fmha_fwd_pp.cuh, fmha_fwd_skv.cuh and
+// attention runs in the kernels of attn_fwd.cuh, attn_fwd_pp.cuh, attn_fwd_skv.cuh and
 // combine.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -14,9 +14,9 @@
 
 #include "../../include/ltxattn.h"
 #include "combine.cuh"
-#include "fmha_fwd.cuh"
-#include "fmha_fwd_pp.cuh"
-#include "fmha_fwd_skv.cuh"
+#include "attn_fwd.cuh"
+#include "attn_fwd_pp.cuh"
+#include "attn_fwd_skv.cuh"
 #include "na3d_fwd.cuh"
 #include "qk_prologue.cuh"
 
@@ -46,6 +46,10 @@ struct Context {
   int* d_status = nullptr;
   EncodeTiledFn encode = nullptr;
   std::map<cudaStream_t, Workspace> workspaces;
+  // held from a split call's workspace lookup through its launches: a grow on one host
+  // thread (stream-ordered free of the old buffer, then a new one) can neither free a
+  // buffer another thread has looked up but not yet launched on, nor race its bookkeeping
+  std::mutex launch_mu;
 };
 
 std::mutex g_mu;
@@ -144,7 +148,7 @@ template <int D, bool kSplit, int kSBuf = 2>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
   dim3 grid(p.n_q_tiles, p.heads, p.batch * p.num_splits);
-  ltx::fmha_fwd_sm100<D, kSplit, kSBuf>
+  ltx::ltx_attn_fwd<D, kSplit, kSBuf>
       <<<grid, FwdSmem<D, kSBuf>::kThreads, FwdSmem<D, kSBuf>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
@@ -154,7 +158,7 @@ template <int D, bool kSplit>
 cudaError_t launch_fwd_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
   dim3 grid((p.n_q_tiles + 1) / 2, p.heads, p.batch * p.num_splits);
-  ltx::fmha_fwd_pp_sm100<D, kSplit><<<grid, ltx::kPPThreads, ltx::PPSmem<D>::kAlloc, stream>>>(
+  ltx::ltx_attn_fwd_pp<D, kSplit><<<grid, ltx::kPPThreads, ltx::PPSmem<D>::kAlloc, stream>>>(
       tq, tk, tv, to, p);
   return cudaGetLastError();
 }
@@ -179,7 +183,7 @@ template <int D, int NKV>
 cudaError_t launch_skv_n(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& to, const FwdParams& p, int grid,
                          cudaStream_t stream) {
-  ltx::fmha_fwd_skv_sm100<D, NKV>
+  ltx::ltx_attn_fwd_skv<D, NKV>
       <<<grid, ltx::kSkvThreads, ltx::SkvSmem<D, NKV>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
@@ -200,45 +204,45 @@ template <int D>
 cudaError_t launch_combine(const FwdParams& p, void* out, cudaStream_t stream) {
   const long long total = (long long)p.batch * p.q_len * p.heads * (D / 4);
   const long long blocks = (total + ltx::kCombineThreads - 1) / ltx::kCombineThreads;
-  ltx::combine_splits<D><<<(unsigned)blocks, ltx::kCombineThreads, 0, stream>>>(
+  ltx::ltx_attn_combine<D><<<(unsigned)blocks, ltx::kCombineThreads, 0, stream>>>(
       p.o_part, p.lse_part, reinterpret_cast<__nv_bfloat16*>(out), p.num_splits, p.batch, p.heads,
       p.q_len, p.n_q_tiles * ltx::kBlockM);
   return cudaGetLastError();
 }
 
 cudaError_t set_smem_limits_dual() {
-  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_sm100<64, true, 1>,
+  cudaError_t e = cudaFuncSetAttribute(ltx::ltx_attn_fwd<64, true, 1>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        FwdSmem<64, 1>::kAlloc);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ltx::fmha_fwd_sm100<64, false, 1>,
+  return cudaFuncSetAttribute(ltx::ltx_attn_fwd<64, false, 1>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64, 1>::kAlloc);
 }
 
 template <int D>
 cudaError_t set_smem_limits() {
-  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_sm100<D, false>,
+  cudaError_t e = cudaFuncSetAttribute(ltx::ltx_attn_fwd<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        FwdSmem<D>::kAlloc);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ltx::fmha_fwd_sm100<D, true>,
+  return cudaFuncSetAttribute(ltx::ltx_attn_fwd<D, true>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<D>::kAlloc);
 }
 
 template <int D>
 cudaError_t set_smem_limits_pp() {
-  cudaError_t e = cudaFuncSetAttribute(ltx::fmha_fwd_pp_sm100<D, false>,
+  cudaError_t e = cudaFuncSetAttribute(ltx::ltx_attn_fwd_pp<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        ltx::PPSmem<D>::kAlloc);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ltx::fmha_fwd_pp_sm100<D, true>,
+  return cudaFuncSetAttribute(ltx::ltx_attn_fwd_pp<D, true>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               ltx::PPSmem<D>::kAlloc);
 }
 
 template <int D, int NKV>
 cudaError_t set_smem_limit_skv() {
-  return cudaFuncSetAttribute(ltx::fmha_fwd_skv_sm100<D, NKV>,
+  return cudaFuncSetAttribute(ltx::ltx_attn_fwd_skv<D, NKV>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               ltx::SkvSmem<D, NKV>::kAlloc);
 }
@@ -251,7 +255,7 @@ cudaError_t set_smem_limits_skv() {
   return e;
 }
 
-__global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
+__global__ void ltx_wait_probe(int* status, unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -265,6 +269,11 @@ __global__ void wait_probe_kernel(int* status, unsigned long long timeout_ns) {
   if (threadIdx.x == 0) ltx::mbar_wait(ltx::smem_u32(&bar), 0, ctl);
   __syncthreads();
 }
+
+// Status word of the allocation-free path on device `dev` (defined with that path below):
+// synchronises `stream`, reads the word and clears it; *ready is false (and nothing is
+// read) when that path was never set up on the device.
+int noalloc_take_status(int dev, cudaStream_t stream, bool* ready);
 
 int read_and_clear_status(Context* c, cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) {
@@ -301,7 +310,7 @@ int launch_prologue(const ltx::PrologueParams& p, cudaStream_t stream) {
     if (resident[dev] == 0) {
       int sms = 0, per_sm = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ltx::qk_norm_rope<CHUNKS, WPR, MIN_CTAS>,
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ltx::ltx_qk_norm_rope<CHUNKS, WPR, MIN_CTAS>,
                                                         ltx::kPrologueWarps * 32, 0) !=
               cudaSuccess ||
           sms < 1 || per_sm < 1) {
@@ -315,7 +324,7 @@ int launch_prologue(const ltx::PrologueParams& p, cudaStream_t stream) {
   constexpr int kRowsPerCta = ltx::PrologueRow<CHUNKS, WPR>::kRowsPerCta;
   const int groups = (2 * p.rows + kRowsPerCta - 1) / kRowsPerCta;
   const unsigned grid = (unsigned)std::min(groups, ctas);
-  ltx::qk_norm_rope<CHUNKS, WPR, MIN_CTAS><<<grid, ltx::kPrologueWarps * 32, 0, stream>>>(p);
+  ltx::ltx_qk_norm_rope<CHUNKS, WPR, MIN_CTAS><<<grid, ltx::kPrologueWarps * 32, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
@@ -329,7 +338,7 @@ constexpr NaShape kNaShapes[] = {{2, 8, 8}, {1, 8, 16}, {4, 4, 8}};
 
 template <int D, int BT, int BY, int BX>
 cudaError_t na_set_smem() {
-  return cudaFuncSetAttribute(ltx::na3d_fwd_sm100<D, BT, BY, BX>,
+  return cudaFuncSetAttribute(ltx::ltx_na3d_fwd<D, BT, BY, BX>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, ltx::NaSmem<D>::kAlloc);
 }
 
@@ -381,9 +390,72 @@ cudaError_t launch_na(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
                       cudaStream_t stream) {
   const long long total = (long long)p.batch * p.heads * p.bricks;
   const int grid = (int)std::min<long long>(total, num_sms);
-  ltx::na3d_fwd_sm100<D, BT, BY, BX>
+  ltx::ltx_na3d_fwd<D, BT, BY, BX>
       <<<grid, ltx::kNaThreads, ltx::NaSmem<D>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
+}
+
+// Rows of key-split partials: [splits][batch][heads][n_q_tiles * 128].
+size_t partial_rows(const FwdParams& p) {
+  return (size_t)p.num_splits * p.batch * p.heads * (size_t)p.n_q_tiles * ltx::kBlockM;
+}
+
+size_t partial_o_bytes(const FwdParams& p, int head_dim) {
+  return partial_rows(p) * (size_t)head_dim * sizeof(float);
+}
+
+// Picks the kernel family and the key-range parts for a call whose sizes are already in
+// `p`; fills p.num_splits and p.tiles_per_split.  num_splits = 0 plans (never above
+// max_splits when that is > 0), >= 1 asks for that many parts (clamped to the key tiles).
+// Returns true for the one-S-buffer, two-CTAs-per-SM variant (head_dim 64, one query tile,
+// a key side longer than two tiles: v2a), whose CTA slots the planner counts twice.
+bool plan_kernel(FwdParams& p, int head_dim, int num_splits, int num_sms, int max_splits) {
+  const bool dual = head_dim == 64 && p.n_kv_tiles > ltx::kSkvMaxKvTiles &&
+                    p.n_q_tiles <= kDualMaxQTiles;
+  // CTAs per key-range part: the two-query-tile kernel takes query tiles in pairs
+  const int q_ctas = (!dual && p.n_q_tiles >= 2) ? (p.n_q_tiles + 1) / 2 : p.n_q_tiles;
+  const int units = q_ctas * p.heads * p.batch;
+  int splits = num_splits > 0 ? std::min(num_splits, p.n_kv_tiles)
+                              : plan_splits(units, p.n_kv_tiles, (dual ? 2 : 1) * num_sms);
+  if (num_splits == 0 && max_splits > 0) splits = std::min(splits, max_splits);
+  p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
+  p.num_splits = (p.n_kv_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty part
+  return dual;
+}
+
+// Launches the planned kernel (and, with key-range parts, the merge into `out`).
+cudaError_t launch_planned(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const CUtensorMap& to, const FwdParams& p, int head_dim, bool dual,
+                           int num_sms, void* out, cudaStream_t stream) {
+  const bool split = p.num_splits > 1;
+  cudaError_t e;
+  if (use_short_kv(p, num_sms)) {
+    return launch_skv(tq, tk, tv, to, p, head_dim, num_sms, stream);
+  } else if (dual) {
+    e = split ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
+              : launch_fwd<64, false, 1>(tq, tk, tv, to, p, stream);
+  } else if (head_dim == 64) {
+    e = split ? launch_attention<64, true>(tq, tk, tv, to, p, stream)
+              : launch_attention<64, false>(tq, tk, tv, to, p, stream);
+  } else {
+    e = split ? launch_attention<128, true>(tq, tk, tv, to, p, stream)
+              : launch_attention<128, false>(tq, tk, tv, to, p, stream);
+  }
+  if (e == cudaSuccess && split)
+    e = head_dim == 64 ? launch_combine<64>(p, out, stream) : launch_combine<128>(p, out, stream);
+  return e;
+}
+
+// Shared-memory limits of every attention kernel on the current device.
+cudaError_t set_smem_limits_all() {
+  cudaError_t e = set_smem_limits<64>();
+  if (e == cudaSuccess) e = set_smem_limits<128>();
+  if (e == cudaSuccess) e = set_smem_limits_pp<64>();
+  if (e == cudaSuccess) e = set_smem_limits_pp<128>();
+  if (e == cudaSuccess) e = set_smem_limits_skv();
+  if (e == cudaSuccess) e = set_smem_limits_dual();
+  if (e == cudaSuccess) e = set_smem_limits_na();
+  return e;
 }
 
 }  // namespace
@@ -411,11 +483,7 @@ int ltxattn_create(void) {
     c->encode = reinterpret_cast<EncodeTiledFn>(fn);
     ok = cudaMalloc(&c->d_status, sizeof(int)) == cudaSuccess &&
          cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
-         set_smem_limits<64>() == cudaSuccess && set_smem_limits<128>() == cudaSuccess &&
-         set_smem_limits_pp<64>() == cudaSuccess && set_smem_limits_pp<128>() == cudaSuccess &&
-         set_smem_limits_skv() == cudaSuccess && set_smem_limits_dual() == cudaSuccess &&
-         set_smem_limits_na() == cudaSuccess &&
-         cudaDeviceSynchronize() == cudaSuccess;
+         set_smem_limits_all() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
     cudaGetLastError();
@@ -449,19 +517,9 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   p.status = c->d_status;
   p.timeout_ns = kDefaultTimeoutNs;
 
-  // head_dim 64 with a long key side and a short query side (v2a): one S buffer per
-  // CTA and two CTAs per SM, so the split planner counts two CTA slots per SM
-  const bool dual = head_dim == 64 && p.n_kv_tiles > ltx::kSkvMaxKvTiles &&
-                    p.n_q_tiles <= kDualMaxQTiles;
-  // CTAs per key-range part: the two-query-tile kernel takes query tiles in pairs
-  const int q_ctas = (!dual && p.n_q_tiles >= 2) ? (p.n_q_tiles + 1) / 2 : p.n_q_tiles;
-  const int units = q_ctas * heads * batch;
-  int splits = num_splits > 0 ? std::min(num_splits, p.n_kv_tiles)
-                              : plan_splits(units, p.n_kv_tiles, (dual ? 2 : 1) * c->num_sms);
-  p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
-  splits = (p.n_kv_tiles + p.tiles_per_split - 1) / p.tiles_per_split;  // no empty part
+  const bool dual = plan_kernel(p, head_dim, num_splits, c->num_sms, 0);
+  const int splits = p.num_splits;
   if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
-  p.num_splits = splits;
   if (splits_used) *splits_used = splits;
 
   CUtensorMap tq, tk, tv, to;
@@ -471,10 +529,11 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
       !encode_bshd(*c, &to, out, q_len, batch, heads, head_dim))
     return LTXATTN_ERR_CUDA;
 
+  std::unique_lock<std::mutex> launch_lock(c->launch_mu, std::defer_lock);
   if (splits > 1) {
-    const size_t rows = (size_t)splits * batch * heads * (size_t)p.n_q_tiles * ltx::kBlockM;
-    const size_t o_bytes = rows * head_dim * sizeof(float);
-    const size_t need = o_bytes + rows * sizeof(float);
+    const size_t o_bytes = partial_o_bytes(p, head_dim);
+    const size_t need = o_bytes + partial_rows(p) * sizeof(float);
+    launch_lock.lock();
     Workspace* ws;
     {
       std::lock_guard<std::mutex> lk(g_mu);
@@ -493,23 +552,7 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
     p.o_part = reinterpret_cast<float*>(ws->ptr);
     p.lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws->ptr) + o_bytes);
   }
-
-  cudaError_t e;
-  if (use_short_kv(p, c->num_sms)) {
-    e = launch_skv(tq, tk, tv, to, p, head_dim, c->num_sms, stream);
-  } else if (dual) {
-    e = splits > 1 ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
-                   : launch_fwd<64, false, 1>(tq, tk, tv, to, p, stream);
-    if (e == cudaSuccess && splits > 1) e = launch_combine<64>(p, out, stream);
-  } else if (head_dim == 64) {
-    e = splits > 1 ? launch_attention<64, true>(tq, tk, tv, to, p, stream)
-                   : launch_attention<64, false>(tq, tk, tv, to, p, stream);
-    if (e == cudaSuccess && splits > 1) e = launch_combine<64>(p, out, stream);
-  } else {
-    e = splits > 1 ? launch_attention<128, true>(tq, tk, tv, to, p, stream)
-                   : launch_attention<128, false>(tq, tk, tv, to, p, stream);
-    if (e == cudaSuccess && splits > 1) e = launch_combine<128>(p, out, stream);
-  }
+  const cudaError_t e = launch_planned(tq, tk, tv, to, p, head_dim, dual, c->num_sms, out, stream);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
@@ -520,11 +563,22 @@ int ltxattn_forward(const void* q, const void* k, const void* v, void* out, int 
                             scale, 0, nullptr, stream);
 }
 
-int ltxattn_check(ltxattn_stream_t stream) {
+int ltxattn_check(ltxattn_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
   int st;
   Context* c = current_context(&st);
-  if (!c) return st;
-  return read_and_clear_status(c, reinterpret_cast<cudaStream_t>(stream));
+  bool noalloc_ready = false;
+  const int st_noalloc = noalloc_take_status(dev, stream, &noalloc_ready);
+  if (!c && !noalloc_ready) return LTXATTN_ERR_NOT_INITIALIZED;
+  const int st_ctx = c ? read_and_clear_status(c, stream) : LTXATTN_OK;
+  for (int want : {(int)LTXATTN_ERR_CUDA, (int)LTXATTN_ERR_DEVICE_TIMEOUT})
+    if (st_ctx == want || st_noalloc == want) return want;
+  return LTXATTN_OK;
 }
 
 int ltxattn_destroy(void) {
@@ -576,7 +630,7 @@ int ltxattn_selftest_wait_timeout(unsigned long long timeout_ns, ltxattn_stream_
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   st = read_and_clear_status(c, stream);  // start from a clean word
   if (st == LTXATTN_ERR_CUDA) return st;
-  wait_probe_kernel<<<1, 32, 0, stream>>>(c->d_status, timeout_ns);
+  ltx_wait_probe<<<1, 32, 0, stream>>>(c->d_status, timeout_ns);
   if (cudaGetLastError() != cudaSuccess) return LTXATTN_ERR_CUDA;
   return read_and_clear_status(c, stream);
 }
@@ -844,7 +898,7 @@ int noalloc_setup(int dev, NoallocDevice** out) {
       return LTXATTN_ERR_CUDA;
     }
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        set_smem_limits<64>() != cudaSuccess || set_smem_limits<128>() != cudaSuccess) {
+        set_smem_limits_all() != cudaSuccess) {
       cudaGetLastError();
       return LTXATTN_ERR_CUDA;
     }
@@ -869,6 +923,33 @@ int noalloc_setup(int dev, NoallocDevice** out) {
 size_t noalloc_bytes(int splits, int batch, int heads, int n_q_tiles, int head_dim) {
   const size_t rows = (size_t)splits * batch * heads * (size_t)n_q_tiles * ltx::kBlockM;
   return kNoallocStatusBytes + rows * (size_t)(head_dim + 1) * sizeof(float);
+}
+
+int noalloc_take_status(int dev, cudaStream_t stream, bool* ready) {
+  *ready = false;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return LTXATTN_OK;
+  unsigned char* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_dev[dev].ready) return LTXATTN_OK;
+    scratch = g_noalloc_dev[dev].scratch;
+  }
+  *ready = true;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  int h = 0;
+  if (cudaMemcpy(&h, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  if (h == ltx::kDevOk) return LTXATTN_OK;
+  if (cudaMemset(scratch, 0, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  return LTXATTN_ERR_DEVICE_TIMEOUT;
 }
 
 }  // namespace
@@ -901,26 +982,24 @@ extern "C" int ltxattn_forward_split_noalloc(const void* q, const void* k, const
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kDefaultTimeoutNs;
 
-  int splits;
-  if (num_splits > 0) {
-    splits = std::min(num_splits, p.n_kv_tiles);
-  } else {
-    splits = plan_splits(p.n_q_tiles * heads * batch, p.n_kv_tiles, d->num_sms);
-    while (splits > 1 && noalloc_bytes(splits, batch, heads, p.n_q_tiles, head_dim) >
-                             LTXATTN_NOALLOC_SCRATCH_BYTES)
-      --splits;
-  }
-  p.tiles_per_split = (p.n_kv_tiles + splits - 1) / splits;
-  splits = (p.n_kv_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  // the most key-range parts whose partials fit in the scratch after the status word; one
+  // part needs no partials at all (the kernel writes the bf16 output itself)
+  const size_t per_split =
+      (size_t)batch * heads * (size_t)p.n_q_tiles * ltx::kBlockM * (size_t)(head_dim + 1) * 4;
+  const size_t fit = (LTXATTN_NOALLOC_SCRATCH_BYTES - kNoallocStatusBytes) / per_split;
+  const int max_splits = (int)std::max<size_t>(1, std::min<size_t>(fit, 1 << 20));
+  const bool dual = plan_kernel(p, head_dim, num_splits, d->num_sms, max_splits);
+  const int splits = p.num_splits;
   if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
-  if (noalloc_bytes(splits, batch, heads, p.n_q_tiles, head_dim) > LTXATTN_NOALLOC_SCRATCH_BYTES)
-    return LTXATTN_ERR_UNSUPPORTED;  // the partials would not fit in the scratch array
-  p.num_splits = splits;
+  if (splits > 1 && noalloc_bytes(splits, batch, heads, p.n_q_tiles, head_dim) >
+                        LTXATTN_NOALLOC_SCRATCH_BYTES)
+    return LTXATTN_ERR_UNSUPPORTED;  // the asked-for partials would not fit in the scratch
 
-  const size_t rows = (size_t)splits * batch * heads * (size_t)p.n_q_tiles * ltx::kBlockM;
   p.status = reinterpret_cast<int*>(d->scratch);
-  p.o_part = reinterpret_cast<float*>(d->scratch + kNoallocStatusBytes);
-  p.lse_part = p.o_part + rows * (size_t)head_dim;
+  if (splits > 1) {
+    p.o_part = reinterpret_cast<float*>(d->scratch + kNoallocStatusBytes);
+    p.lse_part = p.o_part + partial_rows(p) * (size_t)head_dim;
+  }
 
   Context c;  // tensor-map encoder only; nothing in it is allocated
   c.encode = g_noalloc_encode;
@@ -936,13 +1015,6 @@ extern "C" int ltxattn_forward_split_noalloc(const void* q, const void* k, const
     cudaGetLastError();
     return LTXATTN_ERR_CUDA;
   }
-  cudaError_t e;
-  if (head_dim == 64) {
-    e = launch_fwd<64, true>(tq, tk, tv, to, p, stream);
-    if (e == cudaSuccess) e = launch_combine<64>(p, out, stream);
-  } else {
-    e = launch_fwd<128, true>(tq, tk, tv, to, p, stream);
-    if (e == cudaSuccess) e = launch_combine<128>(p, out, stream);
-  }
+  const cudaError_t e = launch_planned(tq, tk, tv, to, p, head_dim, dual, d->num_sms, out, stream);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }

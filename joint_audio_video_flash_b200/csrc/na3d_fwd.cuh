@@ -37,7 +37,7 @@
 // Registers (setmaxnreg): producer/MMA warpgroup 80, softmax 232, epilogue 128.
 #pragma once
 
-#include "fmha_fwd.cuh"
+#include "attn_fwd.cuh"
 
 namespace ltx {
 
@@ -159,7 +159,7 @@ __device__ __forceinline__ uint32_t na_bits(int lo, int hi, int n) {
 
 template <int D, int BT, int BY, int BX>
 __global__ void __launch_bounds__(kNaThreads, 1)
-    na3d_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    ltx_na3d_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const Na3dParams p) {
   static_assert(BT * BY * BX == kBlockM && BX <= 32 && BY <= 32 && BT <= 32, "brick");

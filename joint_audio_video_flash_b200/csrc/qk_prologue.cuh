@@ -143,7 +143,7 @@ __device__ __forceinline__ void prologue_row(const PrologueParams& p, int gr, in
 // MIN_CTAS: CTAs an SM must hold (the register cap; measured per row width, see the launch).
 template <int CHUNKS, int WPR, int MIN_CTAS>
 __global__ void __launch_bounds__(kPrologueWarps * 32, MIN_CTAS)
-    qk_norm_rope(const PrologueParams p) {
+    ltx_qk_norm_rope(const PrologueParams p) {
   static_assert(kPrologueWarps % WPR == 0, "a CTA holds whole rows");
   constexpr int kRowsPerCta = PrologueRow<CHUNKS, WPR>::kRowsPerCta;
   __shared__ float red[2][kPrologueWarps];

@@ -102,6 +102,29 @@ def selftest_wait_timeout(timeout_ns: int = 1_000_000, stream=None) -> int:
                                                       ctypes.c_void_p(_stream_handle(stream))))
 
 
+def _check_attention_tensors(q, k, v, out) -> None:
+    """Checks the library cannot make from raw pointers: bf16, contiguous 4-D BSHD, k and v
+    shaped [batch, kv_len, heads, head_dim] like q, out shaped like q, every tensor on the
+    current CUDA device (the C ABI works on the current device's context).  `out` may be
+    None (checked later, once allocated)."""
+    import torch
+    named = [("q", q), ("k", k), ("v", v)] + ([("out", out)] if out is not None else [])
+    for name, t in named:
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [batch, len, heads, head_dim] tensor")
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{name} is on {t.device}, not on the current device "
+                             f"cuda:{torch.cuda.current_device()}")
+    batch, _, heads, head_dim = q.shape
+    kv_len = k.shape[1]
+    if tuple(k.shape) != (batch, kv_len, heads, head_dim) or v.shape != k.shape:
+        raise ValueError("k and v must be [batch, kv_len, heads, head_dim] matching q")
+    if out is not None and out.shape != q.shape:
+        raise ValueError("out must be shaped like q")
+
+
 def forward(q, k, v, out=None, *, kv_valid_len: int | None = None, scale: float | None = None,
             num_splits: int = 0, stream=None, return_splits: bool = False):
     """O = softmax(scale q k^T, keys < kv_valid_len) v for bf16 BSHD CUDA tensors.
@@ -109,20 +132,12 @@ def forward(q, k, v, out=None, *, kv_valid_len: int | None = None, scale: float 
     q: [B, Lq, H, D]; k, v: [B, Lkv, H, D]; out (optional): [B, Lq, H, D].
     """
     import torch
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
-            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
-        if t.dim() != 4 or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous [batch, len, heads, head_dim] tensor")
+    if out is None:
+        _check_attention_tensors(q, k, v, None)
+        out = torch.empty_like(q)
+    _check_attention_tensors(q, k, v, out)
     batch, q_len, heads, head_dim = q.shape
     kv_len = k.shape[1]
-    if tuple(k.shape) != (batch, kv_len, heads, head_dim) or v.shape != k.shape:
-        raise ValueError("k and v must be [batch, kv_len, heads, head_dim] matching q")
-    if out is None:
-        out = torch.empty_like(q)
-    elif (out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous()
-          or out.device != q.device):
-        raise ValueError("out must be a contiguous bf16 tensor shaped like q on q's device")
     if kv_valid_len is None:
         kv_valid_len = kv_len
     if scale is None:
@@ -143,10 +158,13 @@ def forward_split_noalloc(q, k, v, out, *, kv_valid_len: int | None = None,
 
     For callers that must not let the library allocate (a plugin host that owns all
     device memory, a serving loop with a fixed memory plan, a hard memory quota):
-    the fp32 partials go to the library's built-in 16 MiB scratch array.  ``out`` is
-    required (this call allocates nothing, not even the output).  Returns the raw
-    status; calls whose GPU work overlaps race on the shared scratch.
+    key-split fp32 partials go to the library's built-in 16 MiB scratch array (one key
+    part needs none).  ``out`` is required (this call allocates nothing, not even the
+    output).  Tensors are checked as for ``forward``.  Returns the raw status; calls whose
+    GPU work overlaps race on the shared scratch; ``check()`` reports a kernel wait that
+    ran out in the last such call.
     """
+    _check_attention_tensors(q, k, v, out)
     lib = load()
     fn = lib.ltxattn_forward_split_noalloc
     vp, ci = ctypes.c_void_p, ctypes.c_int

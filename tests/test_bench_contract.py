@@ -71,6 +71,9 @@ def test_gpu_arm_line():
     # four calls per step, one launch each (no key-range parts at these sizes)
     assert d["gpu_launches"] == 4 * d["steps"]
     assert set(d["per_call"]) == {"video_self", "audio_self", "v2a", "a2v"}
+    for name, pc in d["per_call"].items():  # the timed outputs against the oracle
+        par = pc["parity"]
+        assert par["finite"] and par["max_abs"] <= 2e-2 and par["rel_l2"] <= 5e-3, (name, par)
     assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
 
@@ -91,3 +94,27 @@ def test_gpu_arm_line_other_workloads(workload, unit):
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["gpu_launches"] == d["steps"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
+
+
+@pytest.mark.gpu
+def test_gpu_arm_per_config_table():
+    # the headline workload also times every other config and next-row workload on its own,
+    # each with parity against the oracle on sampled rows
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    d = _run(["--steps", "3", "--warmup", "3", "--per-config-steps", "2", "--cpu-seconds", "1"],
+             timeout=1500)
+    assert d["config"]["workload"] == "block768"
+    pc = d["per_config"]
+    assert set(pc) == {"tiny", "video15360_b1", "audio_stream", "longclip", "text_xattn",
+                       "qk_prologue", "na3d_decoder"}
+    pars = [c["parity"] for cfg in pc.values() if "calls" in cfg for c in cfg["calls"].values()]
+    pars += [pc["qk_prologue"]["parity"], pc["na3d_decoder"]["parity"]]
+    pars += [c["parity"] for c in d["per_call"].values()]
+    for par in pars:
+        assert par["finite"] and par["max_abs"] <= 2e-2 and par["rel_l2"] <= 5e-3, par
+    for cfg in pc.values():
+        for c in cfg.get("calls", {"_": cfg}).values():
+            assert c["us_p10"] <= c["us_median"] <= c["us_p90"]
+    assert pc["na3d_decoder"]["density"] > 0 and pc["qk_prologue"]["frac_hbm"] > 0

@@ -334,3 +334,38 @@ def test_bounded_wait_reports_timeout_and_context_survives(oracle):
     q, k, v = synth.make_qkv(1, 130, 300, 2, 64, seed=13)
     got, _ = gpu_run(q, k, v, 300, 0.125)
     assert_parity(got, oracle.attention(q, k, v, 0.125), "after self-test")
+
+
+def test_two_host_threads_share_one_stream(oracle):
+    # two host threads enqueue key-split calls of different workspace sizes on one stream,
+    # so that one thread grows the stream's workspace while the other launches on it
+    import threading
+    cases = [synth.make_qkv(2, 126, 1024 * (i + 2), 4, 64, seed=60 + i, kv_valid=1000 * (i + 2))
+             for i in range(4)]
+    valids = [1000 * (i + 2) for i in range(4)]
+    dev = [[t.cuda() for t in c] for c in cases]
+    outs = [torch.empty_like(d[0]) for d in dev]
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    errors = []
+
+    def worker(idxs):
+        try:
+            torch.cuda.set_device(0)
+            for rep in range(4):
+                for i in idxs:
+                    ltxattn.forward(*dev[i], outs[i], kv_valid_len=valids[i], scale=0.125,
+                                    num_splits=2 + (rep + i) % 4, stream=stream)
+        except Exception as e:  # reported below, on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(ix,)) for ix in ([0, 3], [1, 2])]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    ltxattn.check(stream)
+    for i, (q, k, v) in enumerate(cases):
+        assert_parity(outs[i].cpu(), oracle.attention(q, k, v, 0.125, kv_valid_len=valids[i]),
+                      f"thread case {i}")
