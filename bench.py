@@ -1059,25 +1059,33 @@ def run_prologue(args):
         dist.destroy_process_group()
 
 
-NA_SHAPES = ((2, 8, 8), (1, 8, 16), (4, 4, 8))  # query bricks the library is built for
+# (query brick, key tile) pairs the library is built for, as t x y x x
+NA_SHAPES = (((2, 8, 8), (2, 8, 8)), ((2, 8, 8), (4, 2, 16)), ((1, 8, 16), (1, 8, 16)),
+             ((1, 8, 16), (1, 16, 8)), ((4, 4, 8), (4, 4, 8)), ((4, 4, 8), (4, 2, 16)))
 
 
-def na_key_tiles(grid, window):
-    """128-key tiles the neighbourhood kernel multiplies per (batch, head): the brick
-    shape with the fewest, as the library picks it (counting only; no attention math)."""
+def na_key_tiles(grid, window, with_shape=False):
+    """128-key tiles the neighbourhood kernel multiplies per (batch, head): the shape pair
+    with the fewest, as the library picks it (counting only; no attention math)."""
     def start(i, k, n):
         return min(max(i - k // 2, 0), n - k)
 
-    def axis(n, blk, k):
+    def axis(n, blk, kblk, k):
         tot = 0
         for a0 in range(0, n, blk):
             a1 = min(a0 + blk, n)
             r0, r1 = start(a0, k, n), start(a1 - 1, k, n) + k
-            tot += -(-(r1 - r0) // blk)
+            tot += -(-(r1 - r0) // kblk)
         return tot
 
-    return min(axis(grid[0], sh[0], window[0]) * axis(grid[1], sh[1], window[1])
-               * axis(grid[2], sh[2], window[2]) for sh in NA_SHAPES)
+    best = min((axis(grid[0], qb[0], kb[0], window[0]) * axis(grid[1], qb[1], kb[1], window[1])
+                * axis(grid[2], qb[2], kb[2], window[2]), qb, kb) for qb, kb in NA_SHAPES)
+    return best if with_shape else best[0]
+
+
+def na_kernel_label(grid, window, d):
+    _, qb, kb = na_key_tiles(grid, window, with_shape=True)
+    return f"ltx_na3d_fwd<{d}, query {qb[0]}x{qb[1]}x{qb[2]}, keys {kb[0]}x{kb[1]}x{kb[2]}>"
 
 
 def run_na3d(args):
@@ -1159,7 +1167,7 @@ def run_na3d(args):
         "config": na3d_config(world),
         "roofline": {"bound": "tensor", "achieved": value, "peak": burst, "unit": "TFLOP/s",
                      "frac": value / burst, "traffic": traffic_per_launch("na3d_decoder"),
-                     "kernel": "ltx_na3d_fwd<128, 2, 8, 8>",
+                     "kernel": na_kernel_label(grid, window, d),
                      "issued_tflops": issued_tflops, "issued_frac": issued_tflops / burst,
                      "density": step_flops / issued,
                      "peak_source": f"{peak_src} bf16_tflops (burst)"},
@@ -1182,6 +1190,174 @@ def run_na3d(args):
         dist.destroy_process_group()
 
 
+CP_SEQ, CP_AUDIO, CP_AUDIO_VALID, CP_SEED = 27280, 256, 252, 91
+CP_METRIC = "context-parallel attention TFLOP/s (video self + v2a, long clip)"
+
+
+def cp_config(world):
+    return {"workload": "cp_longclip",
+            "description": "long clip 1280x704x241: video self-attention over 27280 tokens "
+                           "(B2, 32x128) with the sequence sharded over the ranks, and v2a "
+                           "(audio 252->256 queries, 32x64) over the sharded video keys; "
+                           "K/V shards broadcast per source rank, partials merged through "
+                           "their softmax statistics",
+            "l2": "inputs larger than L2", "parallelism": f"cp{world} (sequence sharded)"}
+
+
+def cp_step_flops():
+    b, h = 2, 32
+    return 4.0 * b * h * 128 * CP_SEQ * CP_SEQ + 4.0 * b * h * 64 * CP_AUDIO_VALID * CP_SEQ
+
+
+def run_cp(args):
+    """Context-parallel attention (the row built on ltxattn_forward_partial and
+    ltxattn_combine) at the long-clip size.  Strong scaling: every step is the whole problem,
+    shared by the ranks; with one GPU the process group has one rank (NCCL all the same)."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    from joint_audio_video_flash_b200 import build, cp, ltxattn, synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world == 1:
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    else:
+        dist_setup(args.gpus)
+    build.build()
+    ltxattn.create()
+    b, h, d, da = 2, 32, 128, 64
+    ls = cp.shard_len(CP_SEQ, world)
+    lo, hi = rank * ls, min(CP_SEQ, (rank + 1) * ls)
+
+    def shard(t):
+        out = torch.zeros((t.shape[0], ls, *t.shape[2:]), dtype=t.dtype)
+        if hi > lo:
+            out[:, :hi - lo] = t[:, lo:hi]
+        return out
+
+    # every rank draws the whole problem from the same seeds and keeps its shard
+    vq, vk, vv = synth.make_qkv(b, CP_SEQ, CP_SEQ, h, d, seed=CP_SEED)
+    aq, _, _ = synth.make_qkv(b, CP_AUDIO, 1, h, da, seed=CP_SEED + 1, q_valid=CP_AUDIO_VALID)
+    _, xk, xv = synth.make_qkv(b, 1, CP_SEQ, h, da, seed=CP_SEED + 2)
+    host = [shard(vq), shard(vk), shard(vv), aq, shard(xk), shard(xv)]
+    dq, dk, dv, daq, dxk, dxv = (t.to(dev) for t in host)
+    stream = torch.cuda.current_stream()
+    outs = {}
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        outs["self"] = cp.self_attention(dq, dk, dv, CP_SEQ, None)
+        if ev is not None:
+            ev[1].record(stream)
+        outs["v2a"] = cp.cross_attention(daq, dxk, dxv, CP_SEQ, None)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ltxattn.check()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = device_uuid(dev)
+    with ClockSampler(uuid) as clocks:
+        dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for s_ in range(args.steps):
+            step(evs[s_])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+    ltxattn.check()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    self_us = [e[0].elapsed_time(e[1]) * 1e3 for e in evs]
+    v2a_us = [e[1].elapsed_time(e[2]) * 1e3 for e in evs]
+    step_flops = cp_step_flops()
+    value = step_flops * args.steps / (total_ms * 1e-3) / 1e12
+    # the dominant kernels: this rank's partials over every shard (tensor-bound)
+    own_flops = 4.0 * b * h * d * max(0, hi - lo) * CP_SEQ
+    t_self = statistics.median(self_us)
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = own_flops / (t_self * 1e-6) / 1e12
+    # end to end: this rank's shards up from pinned host memory, both results down
+    pinned = [t.pin_memory() for t in host]
+    dsts = [dq, dk, dv, daq, dxk, dxv]
+    h_self = torch.empty((b, ls, h, d), dtype=torch.bfloat16, pin_memory=True)
+    h_v2a = torch.empty((b, CP_AUDIO, h, da), dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for dst, src in zip(dsts, pinned):
+            dst.copy_(src, non_blocking=True)
+        step()
+        h_self.copy_(outs["self"], non_blocking=True)
+        h_v2a.copy_(outs["v2a"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    line = {
+        "metric": CP_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cp_config(world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                     "frac": achieved / burst, "traffic": None,
+                     "kernel": "ltx_attn_fwd_pp<128, split> over every shard + ltx_attn_combine",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "note": "this rank's video self-attention (partials, exchange waits and "
+                             "merge) timed with CUDA events"},
+        "per_call": {"video_self_cp": dist_stats(self_us), "v2a_cp": dist_stats(v2a_us)},
+        "e2e": {"value": step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host),
+                "d2h_bytes_per_step": h_self.numel() * 2 + h_v2a.numel() * 2,
+                "steps": e2e_steps},
+        "gpu_launches": None,
+        "clocks": clocks.summary(),
+    }
+    # launches per step: one partial per non-empty shard + the merge, and v2a's partial + merge
+    n_shards = sum(1 for r in range(world) if cp.shard_valid(CP_SEQ, world, r) > 0)
+    line["gpu_launches"] = (n_shards + 1 + (1 if hi > lo else 0) + 1) * args.steps
+    if rank == 0 and not args.no_parity:
+        from oracle import oracle
+        rows_s = synth.sample_rows(b, ls, h, 2, seed=CP_SEED, full_heads=())
+        bi, rem = rows_s // (ls * h), rows_s % (ls * h)
+        i, hh = rem // h, rem % h
+        keep = (lo + i) < hi
+        rows_s, bi, i, hh = rows_s[keep], bi[keep], i[keep], hh[keep]
+        full_rows = ((bi * CP_SEQ + lo + i) * h + hh).numpy()
+        ref = oracle.attention(vq, vk, vv, d ** -0.5, rows=full_rows)
+        got = outs["self"].cpu().to(torch.float64).reshape(-1, d)[rows_s].numpy()
+        par = {"video_self_cp": parity_stats(got, ref)}
+        ref2 = oracle.attention(aq, xk, xv, da ** -0.5)
+        par["v2a_cp"] = parity_stats(outs["v2a"].cpu().to(torch.float64).numpy(), ref2)
+        line["parity"] = par
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from joint_audio_video_flash_b200 import workloads
+        calls = [c for c in workloads.configs()["longclip"][1] if c.name in ("video_self", "v2a")]
+        line["cpu_baseline"] = cpu_baseline(calls, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1199,8 +1375,16 @@ def main():
     ap.add_argument("--per-config-steps", type=int, default=10)
     ap.add_argument("--once", action="store_true",
                     help="run each call of the workload once and exit (profiling)")
+    ap.add_argument("--cp", action="store_true",
+                    help="context-parallel attention at the long-clip size (sequence sharded "
+                         "over the ranks; strong scaling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.cp and args.impl != "reference":
+        run_cp(args)
+        return
+    if args.cp:
+        args.workload = "longclip"
     if args.workload in ("qk_prologue", "na3d_decoder") and args.impl == "reference":
         run_reference_other(args)
     elif args.workload == "qk_prologue":

@@ -6,10 +6,12 @@ softmax statistics ("feat(ltx2): tile-parallel video VAE and the two-stage pipel
 commit "Onboard Lightricks LTX-2.5"; "LTX-2: replicate audio stream across Ulysses ranks
 by default", Description).  Two exchange patterns cover the block's attentions:
 
-* self-attention over a sharded sequence (video self): every rank gathers all shards of K
-  and V, computes its own queries' attention over each shard as a partial result (fp32
-  output and base-2 log-sum-exp, ``ltxattn_forward_partial``; its own shard first, while
-  the gathers run) and merges the partials (``ltxattn_combine``);
+* self-attention over a sharded sequence (video self): every rank receives all shards of K
+  and V (one broadcast per source rank), computes its own queries' attention over each
+  shard as a partial result (fp32 output and base-2 log-sum-exp,
+  ``ltxattn_forward_partial``; its own shard first, then each remote shard as soon as it
+  has arrived, while the later ones are still in flight) and merges the partials
+  (``ltxattn_combine``);
 * replicated queries over sharded keys and values (v2a: audio queries, video keys): every
   rank computes the partial over its own shard; the partials and their statistics are
   all-gathered and merged, so every rank ends with the full result.
@@ -19,9 +21,9 @@ exchange: they run locally through ``ltxattn.forward``.
 
 Shards are contiguous, equal ranges of ceil(L / world) tokens, rank r holding tokens
 [r * Ls, min(L, (r + 1) * Ls)), zero-padded to Ls; a rank whose range is empty contributes
-no partial.  The collectives are torch.distributed all-gathers (NCCL between GPUs); every
-step of the attention itself runs in the library's kernels (``backend``, which tests on
-CPU replace).
+no partial.  The collectives are torch.distributed broadcasts and all-gathers (NCCL between
+GPUs); every step of the attention itself runs in the library's kernels (``backend``, which
+tests on CPU replace).
 """
 from __future__ import annotations
 
@@ -67,6 +69,26 @@ def _rows_pad(q_len: int) -> int:
     return -(-int(q_len) // 128) * 128
 
 
+def _post_shards(parts, group):
+    """Every rank's shard, one broadcast per source rank, all posted asynchronously in rank
+    order (the same order on every rank, as collectives require).  `parts` are this rank's
+    tensors of one shard (e.g. its K and V), stacked into slot [rank] of the returned
+    [world, len(parts), *shape] buffer; the other slots receive the other ranks' shards.
+    Returns the buffer and one work handle per source rank."""
+    import torch
+    import torch.distributed as dist
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    buf = torch.empty((world, len(parts), *parts[0].shape), dtype=parts[0].dtype,
+                      device=parts[0].device)
+    for i, t in enumerate(parts):
+        buf[rank, i].copy_(t)
+    works = []
+    for src in range(world):
+        g_src = dist.get_global_rank(group, src) if group is not None else src
+        works.append(dist.broadcast(buf[src], src=g_src, group=group, async_op=True))
+    return buf, works
+
+
 def self_attention(q_local, k_local, v_local, seq_len: int, group, *, scale: float | None = None,
                    backend=None):
     """Attention of this rank's query shard over the whole sharded sequence.
@@ -74,6 +96,11 @@ def self_attention(q_local, k_local, v_local, seq_len: int, group, *, scale: flo
     q_local, k_local, v_local: [B, Ls, H, D], this rank's shard of a sequence of seq_len
     tokens (zero-padded to Ls = ceil(seq_len / world)).  Returns [B, Ls, H, D]; rows past
     the rank's real tokens are not meaningful.
+
+    The shards travel one broadcast per source rank; this rank's own partial runs first,
+    while they are in flight, and the partial over each remote shard is enqueued right
+    after that shard's broadcast (in ring order from this rank), so the transfer of later
+    shards overlaps the attention over earlier ones.
     """
     import torch
     import torch.distributed as dist
@@ -85,24 +112,23 @@ def self_attention(q_local, k_local, v_local, seq_len: int, group, *, scale: flo
         raise ValueError(f"shards must be [B, {shard_len(seq_len, world)}, H, D] on every rank")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     rank = dist.get_rank(group)
-    # the gathers run while this rank's own shard, already local, gives its partial
-    (kb, wk), (vb, wv) = _gather(k_local, group, True), _gather(v_local, group, True)
+    kvb, works = _post_shards((k_local, v_local), group)  # [world, 2, B, Ls, H, D]
     ranks = [r for r in range(world) if shard_valid(seq_len, world, r) > 0]
     rp = _rows_pad(ls)
     o_parts = torch.empty((len(ranks), batch, heads, rp, d), dtype=torch.float32,
                           device=q_local.device)
     lses = torch.empty((len(ranks), batch, heads, rp), dtype=torch.float32,
                        device=q_local.device)
-    if rank in ranks:
-        i = ranks.index(rank)
-        backend.partial(q_local, k_local, v_local, shard_valid(seq_len, world, rank), scale,
-                        o_parts[i], lses[i])
-    wk.wait()
-    wv.wait()
-    for i, r in enumerate(ranks):
+    for s in range(world):
+        r = (rank + s) % world
         if r != rank:
-            backend.partial(q_local, kb[r], vb[r], shard_valid(seq_len, world, r), scale,
+            works[r].wait()  # the stream waits for shard r; the host does not block
+        if r in ranks:
+            i = ranks.index(r)
+            k_r, v_r = (k_local, v_local) if r == rank else (kvb[r, 0], kvb[r, 1])
+            backend.partial(q_local, k_r, v_r, shard_valid(seq_len, world, r), scale,
                             o_parts[i], lses[i])
+    works[rank].wait()  # this rank's own send has read its slot before the buffer goes
     return backend.combine(o_parts, lses, ls)
 
 

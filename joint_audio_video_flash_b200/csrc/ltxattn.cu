@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <map>
 #include <mutex>
+#include <utility>
 
 #include "../../include/ltxattn.h"
 #include "combine.cuh"
@@ -329,53 +330,64 @@ int launch_prologue(const ltx::PrologueParams& p, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- neighbourhood attention
-// Query brick shapes (t x y x x = 128 tokens) the kernel is built for; the host takes the
-// one whose bricks meet the fewest key tiles in total.
+// Query brick and key tile shapes (t x y x x = 128 tokens each) the kernel is built for; the
+// host takes the pair whose bricks meet the fewest key tiles in total.
 struct NaShape {
-  int bt, by, bx;
+  int bt, by, bx;  // query brick
+  int kt, ky, kx;  // key tile
 };
-constexpr NaShape kNaShapes[] = {{2, 8, 8}, {1, 8, 16}, {4, 4, 8}};
+constexpr NaShape kNaShapes[] = {
+    {2, 8, 8, 2, 8, 8}, {2, 8, 8, 4, 2, 16}, {1, 8, 16, 1, 8, 16},
+    {1, 8, 16, 1, 16, 8}, {4, 4, 8, 4, 4, 8}, {4, 4, 8, 4, 2, 16},
+};
+constexpr int kNumNaShapes = (int)(sizeof(kNaShapes) / sizeof(kNaShapes[0]));
 
-template <int D, int BT, int BY, int BX>
+template <int D, int I>
 cudaError_t na_set_smem() {
-  return cudaFuncSetAttribute(ltx::ltx_na3d_fwd<D, BT, BY, BX>,
+  constexpr NaShape s = kNaShapes[I];
+  return cudaFuncSetAttribute(ltx::ltx_na3d_fwd<D, s.bt, s.by, s.bx, s.kt, s.ky, s.kx>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, ltx::NaSmem<D>::kAlloc);
 }
 
-cudaError_t set_smem_limits_na() {
+template <int D, int... I>
+cudaError_t na_set_smem_all(std::integer_sequence<int, I...>) {
   cudaError_t e = cudaSuccess;
-  for (cudaError_t x : {na_set_smem<64, 2, 8, 8>(), na_set_smem<64, 1, 8, 16>(),
-                        na_set_smem<64, 4, 4, 8>(), na_set_smem<128, 2, 8, 8>(),
-                        na_set_smem<128, 1, 8, 16>(), na_set_smem<128, 4, 4, 8>()})
+  for (cudaError_t x : {na_set_smem<D, I>()...})
     if (x != cudaSuccess) e = x;
   return e;
+}
+
+cudaError_t set_smem_limits_na() {
+  const cudaError_t a = na_set_smem_all<64>(std::make_integer_sequence<int, kNumNaShapes>{});
+  const cudaError_t b = na_set_smem_all<128>(std::make_integer_sequence<int, kNumNaShapes>{});
+  return a != cudaSuccess ? a : b;
 }
 
 // Key tiles met by all query bricks of one (batch, head): per axis the sum over bricks of
 // the tiles covering their windows; the axes multiply.
 long long na_tiles_total(const NaShape& b, int t, int y, int x, int kt, int ky, int kx) {
-  auto axis = [](int n, int blk, int k) {
+  auto axis = [](int n, int blk, int kblk, int k) {
     long long sum = 0;
     for (int a0 = 0; a0 < n; a0 += blk) {
       int r0, tiles;
-      ltx::na_key_span(a0, blk, k, n, r0, tiles);
+      ltx::na_key_span(a0, blk, kblk, k, n, r0, tiles);
       sum += tiles;
     }
     return sum;
   };
-  return axis(t, b.bt, kt) * axis(y, b.by, ky) * axis(x, b.bx, kx);
+  return axis(t, b.bt, b.kt, kt) * axis(y, b.by, b.ky, ky) * axis(x, b.bx, b.kx, kx);
 }
 
 // BSHD bf16 tensor over a T x Y x X grid, [batch, T*Y*X, heads, head_dim], seen as a 5-D
 // TMA tensor (heads*head_dim, x, y, t, batch): a box is 64 columns of one head over a
 // bt x by x bx brick of tokens, 128-byte swizzled.
 bool encode_grid(const Context& c, CUtensorMap* map, const void* base, int batch, int t, int y,
-                 int x, int heads, int head_dim, const NaShape& b) {
+                 int x, int heads, int head_dim, int bt, int by, int bx) {
   const cuuint64_t row = (cuuint64_t)heads * head_dim * 2;
   const cuuint64_t dims[5] = {(cuuint64_t)heads * head_dim, (cuuint64_t)x, (cuuint64_t)y,
                               (cuuint64_t)t, (cuuint64_t)batch};
   const cuuint64_t strides[4] = {row, row * x, row * x * y, row * x * y * t};
-  const cuuint32_t box[5] = {64, (cuuint32_t)b.bx, (cuuint32_t)b.by, (cuuint32_t)b.bt, 1};
+  const cuuint32_t box[5] = {64, (cuuint32_t)bx, (cuuint32_t)by, (cuuint32_t)bt, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapL2promotion promo =
       head_dim * 2 >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
@@ -384,15 +396,27 @@ bool encode_grid(const Context& c, CUtensorMap* map, const void* base, int batch
                   promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BT, int BY, int BX>
-cudaError_t launch_na(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const CUtensorMap& to, const ltx::Na3dParams& p, int num_sms,
-                      cudaStream_t stream) {
+template <int D, int I>
+cudaError_t launch_na_shape(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& to, const ltx::Na3dParams& p, int num_sms,
+                            cudaStream_t stream) {
+  constexpr NaShape s = kNaShapes[I];
   const long long total = (long long)p.batch * p.heads * p.bricks;
   const int grid = (int)std::min<long long>(total, num_sms);
-  ltx::ltx_na3d_fwd<D, BT, BY, BX>
+  ltx::ltx_na3d_fwd<D, s.bt, s.by, s.bx, s.kt, s.ky, s.kx>
       <<<grid, ltx::kNaThreads, ltx::NaSmem<D>::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
+}
+
+// The instantiation for shape `shape` (an index into kNaShapes).
+template <int D, int... I>
+cudaError_t launch_na(int shape, const CUtensorMap& tq, const CUtensorMap& tk,
+                      const CUtensorMap& tv, const CUtensorMap& to, const ltx::Na3dParams& p,
+                      int num_sms, cudaStream_t stream, std::integer_sequence<int, I...>) {
+  cudaError_t e = cudaErrorInvalidValue;
+  ((shape == I ? (void)(e = launch_na_shape<D, I>(tq, tk, tv, to, p, num_sms, stream)) : (void)0),
+   ...);
+  return e;
 }
 
 // Rows of key-split partials: [splits][batch][heads][n_q_tiles * 128].
@@ -712,7 +736,7 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
 
   int best = 0;
   long long best_tiles = -1;
-  for (int i = 0; i < (int)(sizeof(kNaShapes) / sizeof(kNaShapes[0])); ++i) {
+  for (int i = 0; i < kNumNaShapes; ++i) {
     const long long t = na_tiles_total(kNaShapes[i], grid_t, grid_y, grid_x, window_t, window_y,
                                        window_x);
     if (best_tiles < 0 || t < best_tiles) {
@@ -739,22 +763,18 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
   p.timeout_ns = kDefaultTimeoutNs;
 
   CUtensorMap tq, tk, tv, to;
-  if (!encode_grid(*c, &tq, q, batch, grid_t, grid_y, grid_x, heads, head_dim, sh) ||
-      !encode_grid(*c, &tk, k, batch, grid_t, grid_y, grid_x, heads, head_dim, sh) ||
-      !encode_grid(*c, &tv, v, batch, grid_t, grid_y, grid_x, heads, head_dim, sh) ||
-      !encode_grid(*c, &to, out, batch, grid_t, grid_y, grid_x, heads, head_dim, sh))
+  // queries and outputs move in query bricks, keys and values in key tiles
+  const int gt = grid_t, gy = grid_y, gx = grid_x;
+  if (!encode_grid(*c, &tq, q, batch, gt, gy, gx, heads, head_dim, sh.bt, sh.by, sh.bx) ||
+      !encode_grid(*c, &tk, k, batch, gt, gy, gx, heads, head_dim, sh.kt, sh.ky, sh.kx) ||
+      !encode_grid(*c, &tv, v, batch, gt, gy, gx, heads, head_dim, sh.kt, sh.ky, sh.kx) ||
+      !encode_grid(*c, &to, out, batch, gt, gy, gx, heads, head_dim, sh.bt, sh.by, sh.bx))
     return LTXATTN_ERR_CUDA;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  cudaError_t e;
-  if (head_dim == 64) {
-    e = best == 0   ? launch_na<64, 2, 8, 8>(tq, tk, tv, to, p, c->num_sms, stream)
-        : best == 1 ? launch_na<64, 1, 8, 16>(tq, tk, tv, to, p, c->num_sms, stream)
-                    : launch_na<64, 4, 4, 8>(tq, tk, tv, to, p, c->num_sms, stream);
-  } else {
-    e = best == 0   ? launch_na<128, 2, 8, 8>(tq, tk, tv, to, p, c->num_sms, stream)
-        : best == 1 ? launch_na<128, 1, 8, 16>(tq, tk, tv, to, p, c->num_sms, stream)
-                    : launch_na<128, 4, 4, 8>(tq, tk, tv, to, p, c->num_sms, stream);
-  }
+  const auto shapes = std::make_integer_sequence<int, kNumNaShapes>{};
+  const cudaError_t e =
+      head_dim == 64 ? launch_na<64>(best, tq, tk, tv, to, p, c->num_sms, stream, shapes)
+                     : launch_na<128>(best, tq, tk, tv, to, p, c->num_sms, stream, shapes);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 

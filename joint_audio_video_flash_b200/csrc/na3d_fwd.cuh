@@ -11,9 +11,11 @@
 //
 // Blocking: a query tile is a brick of BT x BY x BX = 128 tokens (one 5-D TMA box, rows in
 // raster order inside the brick).  The keys any of its queries can see form a box (the
-// union of their windows); it is covered by key tiles that are bricks of the same shape
-// starting at the box's corner (one 5-D TMA box each, zero fill past the grid), so a
-// query brick meets nt * ny * nx key tiles.  The scores of every tile are masked per
+// union of their windows); it is covered by key tiles that are KT x KY x KX bricks of 128
+// keys starting at the box's corner (one 5-D TMA box each, zero fill past the grid), so a
+// query brick meets nt * ny * nx key tiles.  The key tile's shape is chosen apart from the
+// query brick's, to cover the box with as few tiles as possible (a 2 x 8 x 8 brick's box
+// for a 3 x 7 x 7 window, 4 x 14 x 14, takes seven 4 x 2 x 16 tiles but eight 2 x 8 x 8).  The scores of every tile are masked per
 // element against the query row's own window (a bias of 0 or -inf per key column and per
 // (t, y) row of the tile, from three bit masks, one per axis), and a warp skips the
 // exponentials of each 32-key chunk that lies outside all of its rows' windows.
@@ -105,18 +107,19 @@ __host__ __device__ __forceinline__ int na_window_start(int i, int k, int n) {
   return s < 0 ? 0 : (s > n - k ? n - k : s);
 }
 
-// Key box of the query positions [a0, min(a0 + b, n)) on one axis: its first position and
-// the number of b-wide key tiles that cover it.
-__host__ __device__ __forceinline__ void na_key_span(int a0, int b, int k, int n, int& r0,
-                                                     int& tiles) {
-  const int a1 = a0 + b < n ? a0 + b : n;
+// Key box of the query positions [a0, min(a0 + bq, n)) on one axis: its first position and
+// the number of bk-wide key tiles that cover it.
+__host__ __device__ __forceinline__ void na_key_span(int a0, int bq, int bk, int k, int n,
+                                                     int& r0, int& tiles) {
+  const int a1 = a0 + bq < n ? a0 + bq : n;
   r0 = na_window_start(a0, k, n);
   const int r1 = na_window_start(a1 - 1, k, n) + k;
-  tiles = (r1 - r0 + b - 1) / b;
+  tiles = (r1 - r0 + bk - 1) / bk;
 }
 
-// One query brick of one (batch, head) and the key tiles it meets.
-template <int BT, int BY, int BX>
+// One query brick (BT x BY x BX) of one (batch, head) and the key tiles (KT x KY x KX
+// bricks, 128 keys each) that cover its key box.
+template <int BT, int BY, int BX, int KT, int KY, int KX>
 struct NaBrick {
   int b, h;
   int t0, y0, x0;  // query brick origin
@@ -135,18 +138,18 @@ struct NaBrick {
     t0 = it * BT;
     y0 = iy * BY;
     x0 = ix * BX;
-    na_key_span(t0, BT, p.win_t, p.grid_t, rt, nt);
-    na_key_span(y0, BY, p.win_y, p.grid_y, ry, ny);
-    na_key_span(x0, BX, p.win_x, p.grid_x, rx, nx);
+    na_key_span(t0, BT, KT, p.win_t, p.grid_t, rt, nt);
+    na_key_span(y0, BY, KY, p.win_y, p.grid_y, ry, ny);
+    na_key_span(x0, BX, KX, p.win_x, p.grid_x, rx, nx);
     n = nt * ny * nx;
   }
   // origin of key tile j (x fastest)
   __device__ __forceinline__ void key_origin(int j, int& kt, int& ky, int& kx) const {
     const int jx = j % nx;
     const int r = j / nx;
-    kt = rt + (r / ny) * BT;
-    ky = ry + (r % ny) * BY;
-    kx = rx + jx * BX;
+    kt = rt + (r / ny) * KT;
+    ky = ry + (r % ny) * KY;
+    kx = rx + jx * KX;
   }
 };
 
@@ -157,14 +160,16 @@ __device__ __forceinline__ uint32_t na_bits(int lo, int hi, int n) {
   return e > a ? ((0xffffffffu >> (32 - (e - a))) << a) : 0u;
 }
 
-template <int D, int BT, int BY, int BX>
+template <int D, int BT, int BY, int BX, int KT, int KY, int KX>
 __global__ void __launch_bounds__(kNaThreads, 1)
     ltx_na3d_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const Na3dParams p) {
   static_assert(BT * BY * BX == kBlockM && BX <= 32 && BY <= 32 && BT <= 32, "brick");
+  static_assert(KT * KY * KX == kBlockN && KT * KY <= 32 && 32 % KX == 0 && KX % 2 == 0,
+                "key tile: 128 keys, rows of KX keys filling whole 32-key chunks");
   using L = NaSmem<D>;
-  using Brick = NaBrick<BT, BY, BX>;
+  using Brick = NaBrick<BT, BY, BX, KT, KY, KX>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -404,30 +409,30 @@ __global__ void __launch_bounds__(kNaThreads, 1)
           tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
         int kt, ky, kx;
         cur.key_origin(j, kt, ky, kx);
-        const uint32_t mt = na_bits(wt0 - kt, wt0 - kt + p.win_t, BT);
-        const uint32_t my = na_bits(wy0 - ky, wy0 - ky + p.win_y, BY);
-        const uint32_t mx = na_bits(wx0 - kx, wx0 - kx + p.win_x, BX);
+        const uint32_t mt = na_bits(wt0 - kt, wt0 - kt + p.win_t, KT);
+        const uint32_t my = na_bits(wy0 - ky, wy0 - ky + p.win_y, KY);
+        const uint32_t mx = na_bits(wx0 - kx, wx0 - kx + p.win_x, KX);
         // window mask as additive biases (0 inside, -inf outside): one per key column x
         // of the tile and one per (t, y) row of it, two packed adds per pair of scores
-        float2 bx2[BX / 2];
+        float2 bx2[KX / 2];
 #pragma unroll
-        for (int c2 = 0; c2 < BX / 2; ++c2)
+        for (int c2 = 0; c2 < KX / 2; ++c2)
           bx2[c2] = make_float2((mx >> (2 * c2)) & 1u ? 0.0f : -INFINITY,
                                 (mx >> (2 * c2 + 1)) & 1u ? 0.0f : -INFINITY);
         uint32_t rows_in = 0;  // (t, y) rows of the tile inside this query's window
         tmem_ld_wait();
 #pragma unroll
-        for (int r = 0; r < BT * BY; ++r) {
-          const bool in = (mt >> (r / BY)) & (my >> (r % BY)) & 1u;
+        for (int r = 0; r < KT * KY; ++r) {
+          const bool in = (mt >> (r / KY)) & (my >> (r % KY)) & 1u;
           rows_in |= (in ? 1u : 0u) << r;
           const float rb = in ? 0.0f : -INFINITY;
           const float2 rb2 = make_float2(rb, rb);
 #pragma unroll
-          for (int c2 = 0; c2 < BX / 2; ++c2) {
-            float2 v = make_float2(s[r * BX + 2 * c2], s[r * BX + 2 * c2 + 1]);
+          for (int c2 = 0; c2 < KX / 2; ++c2) {
+            float2 v = make_float2(s[r * KX + 2 * c2], s[r * KX + 2 * c2 + 1]);
             v = __fadd2_rn(__fadd2_rn(v, bx2[c2]), rb2);
-            s[r * BX + 2 * c2] = v.x;
-            s[r * BX + 2 * c2 + 1] = v.y;
+            s[r * KX + 2 * c2] = v.x;
+            s[r * KX + 2 * c2 + 1] = v.y;
           }
         }
         const float mx_t = row_max<kBlockN>(s) * sl2;
@@ -464,7 +469,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         for (int c = 0; c < kBlockN / 32; ++c) {
           // a 32-key chunk outside every window of this warp's rows: P = 0 without the
           // exponentials (the MUFU bounds this loop)
-          constexpr int kRowsChunk = 32 / BX;
+          constexpr int kRowsChunk = 32 / KX;
           const uint32_t chunk_rows = (rows_in >> (c * kRowsChunk)) & ((1u << kRowsChunk) - 1u);
           uint32_t pk[16];
           if (__any_sync(0xffffffffu, chunk_rows != 0)) {

@@ -118,3 +118,18 @@ def test_gpu_arm_per_config_table():
         for c in cfg.get("calls", {"_": cfg}).values():
             assert c["us_p10"] <= c["us_median"] <= c["us_p90"]
     assert pc["na3d_decoder"]["density"] > 0 and pc["qk_prologue"]["frac_hbm"] > 0
+
+
+@pytest.mark.gpu
+def test_gpu_arm_context_parallel_line():
+    # context-parallel mode on one GPU: a one-rank NCCL group, the long clip's video self and
+    # v2a through the partial + merge path, with parity against the oracle on sampled rows
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    d = _run(["--cp", "--steps", "2", "--warmup", "3", "--cpu-seconds", "1"], timeout=1500)
+    assert COMMON <= set(d) and d["scaling"] == "strong" and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "cp_longclip" and d["value"] > 0
+    for name, par in d["parity"].items():
+        assert par["finite"] and par["max_abs"] <= 2e-2 and par["rel_l2"] <= 5e-3, (name, par)
+    assert d["gpu_launches"] == 4 * d["steps"]  # one shard: partial + merge, v2a: partial + merge
