@@ -36,6 +36,12 @@
  * stream never launch on a buffer another thread is replacing.  ltxattn_destroy must
  * not run concurrently with other calls on the same device.
  *
+ * Debug build.  Compiled with -DLTXATTN_DEBUG (libltxattn_debug.so), a key-split call puts
+ * canary guard words before and after its fp32 partials, fills the padded rows of every
+ * partial slab with the canary too, and checks all of them on the device after the merge;
+ * an overwritten word is recorded in the device status word and reported by ltxattn_check
+ * as LTXATTN_ERR_WORKSPACE_GUARD.  The release build has none of this.
+ *
  * Errors.  Every entry point returns an ltxattn_status.  Argument checks run on
  * the host, before any CUDA call and before anything is enqueued, so a rejected
  * call has no effect.  Compute calls are asynchronous on `stream` and never
@@ -68,7 +74,10 @@ typedef enum {
   LTXATTN_ERR_MISALIGNED = 3,      /* a tensor base address not 16-byte aligned */
   LTXATTN_ERR_CUDA = 4,            /* a CUDA runtime or driver call failed */
   LTXATTN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel hit its wait limit (see ltxattn_check) */
-  LTXATTN_ERR_NOT_INITIALIZED = 6  /* no context on the current device: call ltxattn_create */
+  LTXATTN_ERR_NOT_INITIALIZED = 6, /* no context on the current device: call ltxattn_create */
+  LTXATTN_ERR_WORKSPACE_GUARD = 7  /* LTXATTN_DEBUG builds only: a key-split call wrote outside
+                                      its partial rows (a guard word or a padded row of the
+                                      workspace was overwritten; see ltxattn_check) */
 } ltxattn_status;
 
 /* Largest sizes accepted (larger values give LTXATTN_ERR_UNSUPPORTED). */
@@ -122,7 +131,8 @@ LTXATTN_API int ltxattn_forward_ex(const void* q, const void* k, const void* v, 
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
- * current device: the context's word (ltxattn_create) and, if
+ * current device (LTXATTN_ERR_WORKSPACE_GUARD for a guard error in the debug
+ * build): the context's word (ltxattn_create) and, if
  * ltxattn_forward_split_noalloc was ever called on this device, that call's own
  * word in its scratch array (read with a plain device-to-host copy; nothing is
  * allocated).  Returns LTXATTN_ERR_DEVICE_TIMEOUT if a kernel recorded a stalled

@@ -8,8 +8,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libltxattn.so")
+DEBUG_LIB = os.path.join(PKG, "libltxattn_debug.so")  # -DLTXATTN_DEBUG: workspace guard words
 SOURCES = ["ltxattn.cu"]
-DEPS = ["ltxattn.cu", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_fwd_skv.cuh", "qk_prologue.cuh", "na3d_fwd.cuh", "combine.cuh", "sm100_ptx.cuh"]
+DEPS = ["ltxattn.cu", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_fwd_skv.cuh", "qk_prologue.cuh",
+        "na3d_fwd.cuh", "combine.cuh", "debug_guard.cuh", "sm100_ptx.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared"]
 
@@ -21,25 +23,28 @@ def _nvcc() -> str:
     return "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", "ltxattn.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/ltxattn.cu (+ headers) into joint_audio_video_flash_b200/libltxattn.so."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile csrc/ltxattn.cu (+ headers) into joint_audio_video_flash_b200/libltxattn.so, or,
+    with debug=True, the guard-word build libltxattn_debug.so (-DLTXATTN_DEBUG)."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *NVCC_FLAGS, *(["-DLTXATTN_DEBUG"] if debug else []), "-o", tmp,
+           *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

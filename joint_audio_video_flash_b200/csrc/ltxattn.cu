@@ -9,12 +9,14 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
 
 #include "../../include/ltxattn.h"
 #include "combine.cuh"
+#include "debug_guard.cuh"
 #include "attn_fwd.cuh"
 #include "attn_fwd_pp.cuh"
 #include "attn_fwd_skv.cuh"
@@ -286,7 +288,7 @@ int read_and_clear_status(Context* c, cudaStream_t stream) {
     return LTXATTN_ERR_CUDA;
   if (h != ltx::kDevOk) {
     if (cudaMemset(c->d_status, 0, sizeof(int)) != cudaSuccess) return LTXATTN_ERR_CUDA;
-    return LTXATTN_ERR_DEVICE_TIMEOUT;
+    return h == ltx::kDevGuard ? LTXATTN_ERR_WORKSPACE_GUARD : LTXATTN_ERR_DEVICE_TIMEOUT;
   }
   return LTXATTN_OK;
 }
@@ -470,6 +472,26 @@ cudaError_t launch_planned(const CUtensorMap& tq, const CUtensorMap& tk, const C
   return e;
 }
 
+#ifdef LTXATTN_DEBUG
+// Checks the guard words and padded rows of the workspace of the split call just enqueued
+// (p.o_part points just past the front guard).  LTXATTN_DEBUG_CORRUPT_GUARD=1 in the
+// environment overwrites one byte of the back guard first, to exercise the detection.
+cudaError_t debug_check_guards(const FwdParams& p, int head_dim, cudaStream_t stream) {
+  const uint32_t* ws = reinterpret_cast<const uint32_t*>(
+      reinterpret_cast<const char*>(p.o_part) - ltx::kGuardBytes);
+  const char* corrupt = std::getenv("LTXATTN_DEBUG_CORRUPT_GUARD");
+  if (corrupt && corrupt[0] == '1') {
+    char* back = reinterpret_cast<char*>(p.lse_part) + partial_rows(p) * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(back + ltx::kGuardBytes - 1, 0x5A, 1, stream);
+    if (e != cudaSuccess) return e;
+  }
+  ltx::ltx_debug_guard_check<<<256, 256, 0, stream>>>(ws, p.num_splits, p.batch, p.heads,
+                                                      p.n_q_tiles * ltx::kBlockM, p.q_len,
+                                                      head_dim, p.status);
+  return cudaGetLastError();
+}
+#endif
+
 // Shared-memory limits of every attention kernel on the current device.
 cudaError_t set_smem_limits_all() {
   cudaError_t e = set_smem_limits<64>();
@@ -554,9 +576,14 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
     return LTXATTN_ERR_CUDA;
 
   std::unique_lock<std::mutex> launch_lock(c->launch_mu, std::defer_lock);
+#ifdef LTXATTN_DEBUG
+  const size_t guard = ltx::kGuardBytes;  // canary words before and after the partials
+#else
+  const size_t guard = 0;
+#endif
   if (splits > 1) {
     const size_t o_bytes = partial_o_bytes(p, head_dim);
-    const size_t need = o_bytes + partial_rows(p) * sizeof(float);
+    const size_t need = o_bytes + partial_rows(p) * sizeof(float) + 2 * guard;
     launch_lock.lock();
     Workspace* ws;
     {
@@ -573,10 +600,16 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
       }
       ws->bytes = need;
     }
-    p.o_part = reinterpret_cast<float*>(ws->ptr);
-    p.lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws->ptr) + o_bytes);
+    p.o_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws->ptr) + guard);
+    p.lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws->ptr) + guard + o_bytes);
+#ifdef LTXATTN_DEBUG
+    if (cudaMemsetAsync(ws->ptr, 0xA5, need, stream) != cudaSuccess) return LTXATTN_ERR_CUDA;
+#endif
   }
-  const cudaError_t e = launch_planned(tq, tk, tv, to, p, head_dim, dual, c->num_sms, out, stream);
+  cudaError_t e = launch_planned(tq, tk, tv, to, p, head_dim, dual, c->num_sms, out, stream);
+#ifdef LTXATTN_DEBUG
+  if (e == cudaSuccess && splits > 1) e = debug_check_guards(p, head_dim, stream);
+#endif
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
 
@@ -600,7 +633,8 @@ int ltxattn_check(ltxattn_stream_t stream_) {
   const int st_noalloc = noalloc_take_status(dev, stream, &noalloc_ready);
   if (!c && !noalloc_ready) return LTXATTN_ERR_NOT_INITIALIZED;
   const int st_ctx = c ? read_and_clear_status(c, stream) : LTXATTN_OK;
-  for (int want : {(int)LTXATTN_ERR_CUDA, (int)LTXATTN_ERR_DEVICE_TIMEOUT})
+  for (int want : {(int)LTXATTN_ERR_CUDA, (int)LTXATTN_ERR_WORKSPACE_GUARD,
+                   (int)LTXATTN_ERR_DEVICE_TIMEOUT})
     if (st_ctx == want || st_noalloc == want) return want;
   return LTXATTN_OK;
 }
@@ -642,6 +676,7 @@ const char* ltxattn_status_string(int status) {
     case LTXATTN_ERR_CUDA: return "LTXATTN_ERR_CUDA";
     case LTXATTN_ERR_DEVICE_TIMEOUT: return "LTXATTN_ERR_DEVICE_TIMEOUT";
     case LTXATTN_ERR_NOT_INITIALIZED: return "LTXATTN_ERR_NOT_INITIALIZED";
+    case LTXATTN_ERR_WORKSPACE_GUARD: return "LTXATTN_ERR_WORKSPACE_GUARD";
     default: return "LTXATTN_UNKNOWN_STATUS";
   }
 }

@@ -19,6 +19,7 @@ namespace ltx {
 enum DeviceStatus : int {
   kDevOk = 0,
   kDevTimeout = 1,
+  kDevGuard = 2,  // a workspace guard word was overwritten (LTXATTN_DEBUG builds only)
 };
 
 struct WaitCtl {

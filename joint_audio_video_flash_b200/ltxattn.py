@@ -14,11 +14,13 @@ import re
 import threading
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libltxattn.so")
+# LTXATTN_DEBUG=1 selects the guard-word build (libltxattn_debug.so, see build.build(debug=True))
+LIB_PATH = os.path.join(_PKG, "libltxattn_debug.so" if os.environ.get("LTXATTN_DEBUG") == "1"
+                        else "libltxattn.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "ltxattn.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_DEVICE_TIMEOUT, \
-    ERR_NOT_INITIALIZED = range(7)
+    ERR_NOT_INITIALIZED, ERR_WORKSPACE_GUARD = range(8)
 
 _lock = threading.Lock()
 _lib = None
@@ -36,7 +38,8 @@ def load() -> ctypes.CDLL:
     with _lock:
         if _lib is None:
             if not os.path.exists(LIB_PATH):
-                raise ImportError(f"{LIB_PATH} is missing: run joint_audio_video_flash_b200.build")
+                raise ImportError(f"{LIB_PATH} is missing: run joint_audio_video_flash_b200.build"
+                                  + (" with debug=True" if LIB_PATH.endswith("_debug.so") else ""))
             lib = ctypes.CDLL(LIB_PATH)
             vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
             lib.ltxattn_create.argtypes = []

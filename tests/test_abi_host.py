@@ -28,11 +28,22 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    names = [ltxattn.status_string(i) for i in range(7)]
+    names = [ltxattn.status_string(i) for i in range(8)]
     assert names[0] == "LTXATTN_OK"
     assert names[5] == "LTXATTN_ERR_DEVICE_TIMEOUT"
-    assert len(set(names)) == 7
+    assert names[7] == "LTXATTN_ERR_WORKSPACE_GUARD"
+    assert len(set(names)) == 8
     assert ltxattn.status_string(99) == "LTXATTN_UNKNOWN_STATUS"
+
+
+def test_debug_build_loads_and_exports_the_same_symbols():
+    # the guard-word build (-DLTXATTN_DEBUG) is a drop-in for the release library
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in ltxattn.header_entry_points():
+        assert hasattr(dbg, name), name
+    dbg.ltxattn_status_string.restype = ctypes.c_char_p
+    assert dbg.ltxattn_status_string(7) == b"LTXATTN_ERR_WORKSPACE_GUARD"
 
 
 # fake, never dereferenced device addresses: validation fails before any CUDA call
