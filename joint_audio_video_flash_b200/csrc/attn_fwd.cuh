@@ -60,6 +60,9 @@ struct FwdParams {
 // warps in the first warpgroup, which hands registers to the softmax warpgroup), three K
 // and two V stages, so that two CTAs share an SM and interleave their
 // QK -> softmax -> PV chains (head_dim 64 only: shared memory and registers fit twice).
+// P has its own 64 columns there (S [0,128), P [128,192), O [192,256)), so QK of the next
+// key tile is issued as soon as the softmax has read S into registers and runs during the
+// exponentials; the softmax writes P(j) once PV(j-1) has read P(j-1).
 template <int D, int kSBuf = 2>
 struct FwdSmem {
   static_assert(kSBuf == 2 || (kSBuf == 1 && D == 64), "S buffers");
@@ -86,7 +89,8 @@ struct FwdSmem {
   static constexpr int bVE = bVF + kVStages;
   static constexpr int bSF = bVE + kVStages;  // kSBuf
   static constexpr int bPF = bSF + 2;        // kSBuf
-  static constexpr int bOD = bPF + 2;        // O updated by a PV
+  static constexpr int bSE = bPF + 2;        // kSBuf == 1: S read into registers (4 warps)
+  static constexpr int bOD = bSE + 1;        // O updated by a PV
   static constexpr int bOF = bOD + 1;        // final PV done
   static constexpr int bDrain = bOF + 1;     // abort-path drain
   static constexpr int kNumBars = bDrain + 1;
@@ -96,7 +100,8 @@ struct FwdSmem {
   static constexpr int kRaw = ((kUsed + 1024 + 1023) / 1024) * 1024;
   static constexpr int kAlloc =
       kSBuf == 1 ? kRaw : (kRaw > kMinSmemFor1Cta ? kRaw : kMinSmemFor1Cta);
-  static constexpr int kColO = 128 * kSBuf;
+  static constexpr int kColP = 128;                    // kSBuf == 1: P's own columns
+  static constexpr int kColO = kSBuf == 1 ? 192 : 256;
   static constexpr uint32_t kTmemCols = kSBuf == 1 ? 256 : 512;
   static_assert(kSBuf == 2 || 2 * kAlloc <= 227 * 1024, "two CTAs per SM");
 };
@@ -144,6 +149,49 @@ __device__ __forceinline__ void exp2_pack16(const float* s, float2 sc2, float2 n
   for (int x = 0; x < 16; ++x) {
     const float2 a = __ffma2_rn(make_float2(s[2 * x], s[2 * x + 1]), sc2, nm2);
     const float2 e = make_float2(ex2(a.x), ex2(a.y));
+    if (x & 1)
+      lb = __fadd2_rn(lb, e);
+    else
+      la = __fadd2_rn(la, e);
+    pk[x] = pack_bf16x2(e.x, e.y);
+  }
+}
+
+// 2^x for a pair on the FMA pipe (no MUFU): Cody-Waite range reduction x = j + f, j the
+// nearest integer (adding 1.5 * 2^23 leaves j in the low mantissa bits) and f in [-1/2, 1/2];
+// 2^f from a cubic whose coefficients come from a Remez exchange for minimax relative error
+// on that interval (7.5e-5, far below the bf16 rounding of P); 2^j is added into the exponent
+// field.  x is clamped below at -126 (the result, <= 2^-126, is zero next to any row sum).
+// Valid for x <= 127.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.055171669f;
+  x = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  // the low 9 bits of t's pattern hold j (two's complement); shifted into the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// exp2_pack16 with every kPolyEvery-th pair of scores (kPolyEvery > 0) exponentiated on the
+// FMA pipe instead of the MUFU, which the exponentials otherwise saturate (one MUFU op per
+// score against 512 tensor FLOPs per score at head_dim 128).  Only for tiles without masked
+// keys: the FMA path gives 2^-126, not 0, for -inf.
+template <int kPolyEvery>
+__device__ __forceinline__ void exp2_pack16_mix(const float* s, float2 sc2, float2 nm2,
+                                                float2& la, float2& lb, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int x = 0; x < 16; ++x) {
+    const float2 a = __ffma2_rn(make_float2(s[2 * x], s[2 * x + 1]), sc2, nm2);
+    constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
+    const float2 e = (kPolyEvery > 0 && x % kEvery == kEvery - 1)
+                         ? exp2_fma2(a)
+                         : make_float2(ex2(a.x), ex2(a.y));
     if (x & 1)
       lb = __fadd2_rn(lb, e);
     else
@@ -201,8 +249,9 @@ __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::bSF + s), 1);
-      mbar_init(bar(L::bPF + s), kBlockM);
+      mbar_init(bar(L::bPF + s), 4);  // one arrival per softmax warp
     }
+    mbar_init(bar(L::bSE), 4);
     mbar_init(bar(L::bOD), 1);
     mbar_init(bar(L::bOF), 1);
     mbar_init(bar(L::bDrain), 1);
@@ -289,25 +338,22 @@ __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
         if (!mbar_wait(bar(L::bVF + st), (uint32_t)(t / L::kVStages) & 1u, ctl)) return false;
         tc_fence_after();
         const uint32_t v_off = (uint32_t)st * L::kTileBytes;
+        // P: its own columns with one S buffer, else packed over the S buffer it came from
+        const uint32_t p_col = kSBuf == 1 ? (uint32_t)L::kColP : (uint32_t)sb * 128;
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
           // B = V tile, N = D (MN-major: d contiguous), K = 16 keys starting at kk*16
-          umma_ts(tmem + L::kColO, tmem + sb * 128 + kk * 8, dv.at(v_off + kk * 16 * 128),
+          umma_ts(tmem + L::kColO, tmem + p_col + kk * 8, dv.at(v_off + kk * 16 * 128),
                   idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(L::bVE + st));
         umma_commit(bar(L::bOD));
         return true;
       };
-      for (int j = 0; j < n && ok; ++j) {
-        if (kSBuf == 1 && j >= 1) {
-          // P(j-1) sits in the only S buffer: its PV goes before QK(j) overwrites it
-          ok = pv(j - 1);
-          if (!ok) break;
-        }
+      // S(j) = Q K_j^T into S buffer j % kSBuf
+      auto qk = [&](int j) -> bool {
         const int st = j % L::kKStages;
-        ok = mbar_wait(bar(L::bKF + st), (uint32_t)(j / L::kKStages) & 1u, ctl);
-        if (!ok) break;
+        if (!mbar_wait(bar(L::bKF + st), (uint32_t)(j / L::kKStages) & 1u, ctl)) return false;
         tc_fence_after();
         const int sb = j % kSBuf;
         const uint32_t k_off = (uint32_t)st * L::kTileBytes;
@@ -319,9 +365,23 @@ __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
         issued = true;
         umma_commit(bar(L::bSF + sb));
         umma_commit(bar(L::bKE + st));
-        if (kSBuf == 2 && j >= 1) ok = pv(j - 1);
+        return true;
+      };
+      if constexpr (kSBuf == 1) {
+        // QK(j+1) needs only the softmax to have read S(j) (P has its own columns), so it
+        // runs during the exponentials of tile j; PV(j) follows when P(j) is published
+        ok = ok && qk(0);
+        for (int j = 0; j < n && ok; ++j) {
+          if (j + 1 < n) ok = mbar_wait(bar(L::bSE), (uint32_t)j & 1u, ctl) && qk(j + 1);
+          ok = ok && pv(j);
+        }
+      } else {
+        for (int j = 0; j < n && ok; ++j) {
+          ok = qk(j);
+          if (ok && j >= 1) ok = pv(j - 1);
+        }
+        if (ok) ok = pv(n - 1);
       }
-      if (ok) ok = pv(n - 1);
       if (ok) {
         umma_commit(bar(L::bOF));
       } else if (issued) {
@@ -355,6 +415,12 @@ __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
       for (int c = 0; c < kBlockN / 32; ++c)
         tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
       tmem_ld_wait();
+      if constexpr (kSBuf == 1) {
+        // S(j) is in registers: QK(j+1) may overwrite it (one arrival per warp)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::bSE));
+      }
       if (lim < kBlockN) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
@@ -389,15 +455,26 @@ __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
       const float2 nm2 = make_float2(-m_run, -m_run);
       const float2 sc2 = make_float2(sl2, sl2);
       float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
+      uint32_t tP = tS;  // P packed over the S buffer it came from ...
+      if constexpr (kSBuf == 1) {
+        // ... or in its own columns, free once PV(j-1) has read P(j-1)
+        tP = trow + L::kColP;
+        if (j >= 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOD), (uint32_t)(j - 1) & 1u, ctl));
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
 #pragma unroll
       for (int c = 0; c < kBlockN / 32; ++c) {
         uint32_t pk[16];
         exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
-        tmem_st16(tS + c * 16, pk);
+        tmem_st16(tP + c * 16, pk);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::bPF + sb));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::bPF + sb));
       l_run += (la.x + la.y) + (lb.x + lb.y);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOF), 0, ctl));

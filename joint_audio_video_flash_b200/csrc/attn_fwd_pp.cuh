@@ -36,6 +36,9 @@ static_assert(128 * kPPRegsProducer + 256 * kPPRegsSoftmax <= kPPThreads * kPPRe
 // the PV of the first parts overlaps the exponentials of the later ones
 constexpr int kPPParts = 2;
 static_assert(kPPParts == 2 || kPPParts == 4, "P parts");
+// Every kPPPolyEvery-th pair of scores of a full key tile is exponentiated on the FMA pipe
+// (exp2_fma2) rather than the MUFU; 0 = all on the MUFU.
+constexpr int kPPPolyEvery = 0;
 
 template <int D>
 struct PPSmem {
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       mbar_init(bar(L::bQF + g), 1);
       mbar_init(bar(L::bSF + g), 1);
       for (int part = 0; part < kPPParts; ++part)  // P keys of one part of tile g
-        mbar_init(bar(L::bPF + part * 2 + g), kBlockM);
+        mbar_init(bar(L::bPF + part * 2 + g), 4);  // one arrival per softmax warp
       mbar_init(bar(L::bOF + g), 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
@@ -318,6 +321,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       // published to the MMA warp in kPPParts key parts so the PV of the first parts
       // overlaps the exponentials of the later ones
       float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
+      [[maybe_unused]] const bool full_tile = kv0 + kBlockN <= p.kv_valid;
 #pragma unroll
       for (int part = 0; part < kPPParts; ++part) {
         constexpr int kChunks = kBlockN / 32 / kPPParts;  // 32-key chunks per part
@@ -325,12 +329,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int c = 0; c < kChunks; ++c) {
           const int ch = part * kChunks + c;
           uint32_t pk[16];
-          exp2_pack16(&s[ch * 32], sc2, nm2, la, lb, pk);
+          if (kPPPolyEvery > 0 && full_tile)
+            exp2_pack16_mix<kPPPolyEvery>(&s[ch * 32], sc2, nm2, la, lb, pk);
+          else
+            exp2_pack16(&s[ch * 32], sc2, nm2, la, lb, pk);
           tmem_st16(trow + colS + ch * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::bPF + part * 2 + g));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::bPF + part * 2 + g));
       }
       l_run += (la.x + la.y) + (lb.x + lb.y);
     }

@@ -141,9 +141,9 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(bar(L::bSF + b), 1);
-      mbar_init(bar(L::bPF + b), kBlockM);
+      mbar_init(bar(L::bPF + b), 4);  // one arrival per softmax warp
       mbar_init(bar(L::bOF + b), 1);
-      mbar_init(bar(L::bTF + b), kBlockM);
+      mbar_init(bar(L::bTF + b), 4);  // one arrival per epilogue warp
     }
     mbar_init(bar(L::bDrain), 1);
     *abort_flag = (*reinterpret_cast<volatile int*>(p.status) != kDevOk) ? 1 : 0;
@@ -387,7 +387,8 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       row_sum[bf * kBlockM + row] = (la.x + la.y) + (lb.x + lb.y);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::bPF + bf));  // P in TMEM and l in shared memory
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::bPF + bf));  // P in TMEM and l in shared memory
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -425,7 +426,8 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
         tmem_ld_wait();
         if (bx == L::kBoxes - 1) {
           tc_fence_before();
-          mbar_arrive(bar(L::bTF + bf));  // S/P/O of this buffer and its l may be reused
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(L::bTF + bf));  // S/P/O and l of this buffer are free
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {  // 8 chunks of 16 bytes = 64 bf16
