@@ -62,7 +62,8 @@ struct FwdParams {
 // QK -> softmax -> PV chains (head_dim 64 only: shared memory and registers fit twice).
 // P has its own 64 columns there (S [0,128), P [128,192), O [192,256)), so QK of the next
 // key tile is issued as soon as the softmax has read S into registers and runs during the
-// exponentials; the softmax writes P(j) once PV(j-1) has read P(j-1).
+// exponentials; the softmax computes P(j) in registers and stores it once PV(j-1) has read
+// P(j-1).
 template <int D, int kSBuf = 2>
 struct FwdSmem {
   static_assert(kSBuf == 2 || (kSBuf == 1 && D == 64), "S buffers");
@@ -149,49 +150,6 @@ __device__ __forceinline__ void exp2_pack16(const float* s, float2 sc2, float2 n
   for (int x = 0; x < 16; ++x) {
     const float2 a = __ffma2_rn(make_float2(s[2 * x], s[2 * x + 1]), sc2, nm2);
     const float2 e = make_float2(ex2(a.x), ex2(a.y));
-    if (x & 1)
-      lb = __fadd2_rn(lb, e);
-    else
-      la = __fadd2_rn(la, e);
-    pk[x] = pack_bf16x2(e.x, e.y);
-  }
-}
-
-// 2^x for a pair on the FMA pipe (no MUFU): Cody-Waite range reduction x = j + f, j the
-// nearest integer (adding 1.5 * 2^23 leaves j in the low mantissa bits) and f in [-1/2, 1/2];
-// 2^f from a cubic whose coefficients come from a Remez exchange for minimax relative error
-// on that interval (7.5e-5, far below the bf16 rounding of P); 2^j is added into the exponent
-// field.  x is clamped below at -126 (the result, <= 2^-126, is zero next to any row sum).
-// Valid for x <= 127.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.055171669f;
-  x = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  p = __ffma2_rn(p, f, make_float2(c1, c1));
-  p = __ffma2_rn(p, f, make_float2(c0, c0));
-  // the low 9 bits of t's pattern hold j (two's complement); shifted into the exponent field
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// exp2_pack16 with every kPolyEvery-th pair of scores (kPolyEvery > 0) exponentiated on the
-// FMA pipe instead of the MUFU, which the exponentials otherwise saturate (one MUFU op per
-// score against 512 tensor FLOPs per score at head_dim 128).  Only for tiles without masked
-// keys: the FMA path gives 2^-126, not 0, for -inf.
-template <int kPolyEvery>
-__device__ __forceinline__ void exp2_pack16_mix(const float* s, float2 sc2, float2 nm2,
-                                                float2& la, float2& lb, uint32_t (&pk)[16]) {
-#pragma unroll
-  for (int x = 0; x < 16; ++x) {
-    const float2 a = __ffma2_rn(make_float2(s[2 * x], s[2 * x + 1]), sc2, nm2);
-    constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
-    const float2 e = (kPolyEvery > 0 && x % kEvery == kEvery - 1)
-                         ? exp2_fma2(a)
-                         : make_float2(ex2(a.x), ex2(a.y));
     if (x & 1)
       lb = __fadd2_rn(lb, e);
     else
@@ -455,21 +413,28 @@ __global__ void __launch_bounds__(FwdSmem<D, kSBuf>::kThreads, 3 - kSBuf)
       const float2 nm2 = make_float2(-m_run, -m_run);
       const float2 sc2 = make_float2(sl2, sl2);
       float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
-      uint32_t tP = tS;  // P packed over the S buffer it came from ...
       if constexpr (kSBuf == 1) {
-        // ... or in its own columns, free once PV(j-1) has read P(j-1)
-        tP = trow + L::kColP;
+        // P has its own columns, which PV(j-1) may still be reading: every exponential
+        // first (P packed in registers), then the wait for that PV, then the stores, so the
+        // exponentials overlap PV(j-1) instead of waiting behind it
+        uint32_t pk[kBlockN / 32][16];
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk[c]);
         if (j >= 1) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOD), (uint32_t)(j - 1) & 1u, ctl));
           if (!ok) break;
           tc_fence_after();
         }
-      }
 #pragma unroll
-      for (int c = 0; c < kBlockN / 32; ++c) {
-        uint32_t pk[16];
-        exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
-        tmem_st16(tP + c * 16, pk);
+        for (int c = 0; c < kBlockN / 32; ++c) tmem_st16(trow + L::kColP + c * 16, pk[c]);
+      } else {
+        // P packed over the S buffer it came from
+#pragma unroll
+        for (int c = 0; c < kBlockN / 32; ++c) {
+          uint32_t pk[16];
+          exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+          tmem_st16(tS + c * 16, pk);
+        }
       }
       tmem_st_wait();
       tc_fence_before();

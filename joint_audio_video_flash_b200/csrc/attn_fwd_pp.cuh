@@ -36,9 +36,6 @@ static_assert(128 * kPPRegsProducer + 256 * kPPRegsSoftmax <= kPPThreads * kPPRe
 // the PV of the first parts overlaps the exponentials of the later ones
 constexpr int kPPParts = 2;
 static_assert(kPPParts == 2 || kPPParts == 4, "P parts");
-// Every kPPPolyEvery-th pair of scores of a full key tile is exponentiated on the FMA pipe
-// (exp2_fma2) rather than the MUFU; 0 = all on the MUFU.
-constexpr int kPPPolyEvery = 0;
 
 template <int D>
 struct PPSmem {
@@ -321,7 +318,6 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       // published to the MMA warp in kPPParts key parts so the PV of the first parts
       // overlaps the exponentials of the later ones
       float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
-      [[maybe_unused]] const bool full_tile = kv0 + kBlockN <= p.kv_valid;
 #pragma unroll
       for (int part = 0; part < kPPParts; ++part) {
         constexpr int kChunks = kBlockN / 32 / kPPParts;  // 32-key chunks per part
@@ -329,10 +325,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int c = 0; c < kChunks; ++c) {
           const int ch = part * kChunks + c;
           uint32_t pk[16];
-          if (kPPPolyEvery > 0 && full_tile)
-            exp2_pack16_mix<kPPPolyEvery>(&s[ch * 32], sc2, nm2, la, lb, pk);
-          else
-            exp2_pack16(&s[ch * 32], sc2, nm2, la, lb, pk);
+          exp2_pack16(&s[ch * 32], sc2, nm2, la, lb, pk);
           tmem_st16(trow + colS + ch * 16, pk);
         }
         tmem_st_wait();

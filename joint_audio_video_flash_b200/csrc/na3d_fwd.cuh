@@ -386,8 +386,6 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     const float2 sc2 = make_float2(sl2, sl2);
     bool ok = !*abort_flag;
     int g = 0;
-    bool pre = false;  // the scores of tile g are already loaded (issued during tile g - 1)
-    float s[kBlockN];
     Brick cur;
     for (int i = 0; i < cnt && ok; ++i) {
       cur.init(unit(i), p);
@@ -401,21 +399,14 @@ __global__ void __launch_bounds__(kNaThreads, 1)
       float l_run = 0.0f;
       for (int j = 0; j < cur.n && ok; ++j, ++g) {
         const int sb = g & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(g >> 1) & 1u, ctl));
+        if (!ok) break;
+        tc_fence_after();
         const uint32_t tS = tlane + sb * 128;
-        if (!pre) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(g >> 1) & 1u, ctl));
-          if (!ok) break;
-          tc_fence_after();
+        float s[kBlockN];
 #pragma unroll
-          for (int c = 0; c < kBlockN / 32; ++c)
-            tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-        }
-        // the next tile (of this brick or the next one): if its scores are already in the
-        // other S buffer, each 32-key chunk of them is loaded into the registers the current
-        // tile's chunk leaves free once its exponentials are out, so the next tile's load
-        // waits behind this tile's exponentials instead of after them
-        const bool has_next = j + 1 < cur.n || i + 1 < cnt;
-        const uint32_t tS_next = tlane + (sb ^ 1) * 128;
+        for (int c = 0; c < kBlockN / 32; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
         int kt, ky, kx;
         cur.key_origin(j, kt, ky, kx);
         const uint32_t mt = na_bits(wt0 - kt, wt0 - kt + p.win_t, KT);
@@ -474,10 +465,6 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         const float2 nm2 = make_float2(-m_use, -m_use);
         float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
         if (mx == 0) rows_in = 0;
-        // non-blocking: the next tile's scores are complete (never waits here)
-        pre = has_next && __all_sync(0xffffffffu, mbar_try_wait(bar(L::bSF + (sb ^ 1)),
-                                                                (uint32_t)((g + 1) >> 1) & 1u));
-        if (pre) tc_fence_after();
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
           // a 32-key chunk outside every window of this warp's rows: P = 0 without the
@@ -492,7 +479,6 @@ __global__ void __launch_bounds__(kNaThreads, 1)
             for (int x = 0; x < 16; ++x) pk[x] = 0u;
           }
           tmem_st16(tS + c * 16, pk);
-          if (pre) tmem_ld32(tS_next + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
         }
         tmem_st_wait();
         tc_fence_before();
