@@ -182,12 +182,13 @@ bool use_short_kv(const FwdParams& p, int num_sms) {
          (long long)p.batch * p.heads * p.n_q_tiles > num_sms;
 }
 
-template <int D, int NKV>
+template <int D, int NKV, bool kTileKV = false>
 cudaError_t launch_skv_n(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& to, const FwdParams& p, int grid,
                          cudaStream_t stream) {
-  ltx::ltx_attn_fwd_skv<D, NKV>
-      <<<grid, ltx::kSkvThreads, ltx::SkvSmem<D, NKV>::kAlloc, stream>>>(tq, tk, tv, to, p);
+  ltx::ltx_attn_fwd_skv<D, NKV, kTileKV>
+      <<<grid, ltx::kSkvThreads, ltx::SkvSmem<D, NKV, kTileKV>::kAlloc, stream>>>(tq, tk, tv,
+                                                                                 to, p);
   return cudaGetLastError();
 }
 
@@ -196,8 +197,10 @@ cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        cudaStream_t stream) {
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
   const int grid = (int)std::min<long long>(total, num_sms);
+  // head_dim 64, one key tile (a2v): per-unit K/V and the strided (batch, query tile, head)
+  // walk, so that the tiles in flight cover whole token rows of q and out
   if (head_dim == 64)
-    return p.n_kv_tiles == 1 ? launch_skv_n<64, 1>(tq, tk, tv, to, p, grid, stream)
+    return p.n_kv_tiles == 1 ? launch_skv_n<64, 1, true>(tq, tk, tv, to, p, grid, stream)
                              : launch_skv_n<64, 2>(tq, tk, tv, to, p, grid, stream);
   return p.n_kv_tiles == 1 ? launch_skv_n<128, 1>(tq, tk, tv, to, p, grid, stream)
                            : launch_skv_n<128, 2>(tq, tk, tv, to, p, grid, stream);
@@ -243,15 +246,16 @@ cudaError_t set_smem_limits_pp() {
                               ltx::PPSmem<D>::kAlloc);
 }
 
-template <int D, int NKV>
+template <int D, int NKV, bool kTileKV = false>
 cudaError_t set_smem_limit_skv() {
-  return cudaFuncSetAttribute(ltx::ltx_attn_fwd_skv<D, NKV>,
+  return cudaFuncSetAttribute(ltx::ltx_attn_fwd_skv<D, NKV, kTileKV>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              ltx::SkvSmem<D, NKV>::kAlloc);
+                              ltx::SkvSmem<D, NKV, kTileKV>::kAlloc);
 }
 
 cudaError_t set_smem_limits_skv() {
   cudaError_t e = set_smem_limit_skv<64, 1>();
+  if (e == cudaSuccess) e = set_smem_limit_skv<64, 1, true>();
   if (e == cudaSuccess) e = set_smem_limit_skv<64, 2>();
   if (e == cudaSuccess) e = set_smem_limit_skv<128, 1>();
   if (e == cudaSuccess) e = set_smem_limit_skv<128, 2>();
