@@ -527,7 +527,6 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       fence_proxy_async_smem();
       named_bar_sync(1, kBlockM);
       if (leader) {
-#pragma unroll
         int sh = cur.h, sqt = cur.qt, sbat = cur.b;
         if constexpr (kTileKV) {
           SkvUnit u;
@@ -536,6 +535,7 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
           sqt = u.qt;
           sbat = u.b;
         }
+#pragma unroll
         for (int bx = 0; bx < L::kBoxes; ++bx)
           tma_store_4d(&tm_o, sbase + L::kStage + sb * L::kTileBytes + bx * L::kBoxBytes,
                        bx * 64, sh, sqt * kBlockM, sbat);

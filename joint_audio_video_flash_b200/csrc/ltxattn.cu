@@ -18,6 +18,7 @@
 #include "combine.cuh"
 #include "debug_guard.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_pair.cuh"
 #include "attn_fwd_pp.cuh"
 #include "attn_fwd_skv.cuh"
 #include "na3d_fwd.cuh"
@@ -95,12 +96,12 @@ int validate(const void* q, const void* k, const void* v, void* out, int q_len, 
 // BSHD bf16 tensor [batch, len, heads, head_dim] seen as a 4-D TMA tensor
 // (d, h, s, b) with a 64-column x 128-row box and the 128-byte swizzle.
 bool encode_bshd(const Context& c, CUtensorMap* map, const void* base, int len, int batch,
-                 int heads, int head_dim) {
+                 int heads, int head_dim, int box_rows = ltx::kBlockM) {
   const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)heads, (cuuint64_t)len,
                               (cuuint64_t)batch};
   const cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)heads * head_dim * 2,
                                  (cuuint64_t)len * heads * head_dim * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)ltx::kBlockM, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   // L2 fetch granule = one (token, head) row: a 256-byte promotion of a 128-byte row
   // would also fetch the next head's row, which a head-ordered walk reads much later
@@ -453,13 +454,34 @@ bool plan_kernel(FwdParams& p, int head_dim, int num_splits, int num_sms, int ma
   return dual;
 }
 
-// Launches the planned kernel (and, with key-range parts, the merge into `out`).
+// Query sides of at least this many 128-row tiles at head_dim 128 (unsplit) run on CTA pairs.
+constexpr int kPairMinQTiles = 8;
+
+bool use_pair(const FwdParams& p, int head_dim, int num_sms) {
+  return head_dim == 128 && p.num_splits == 1 && p.n_q_tiles >= kPairMinQTiles &&
+         !use_short_kv(p, num_sms);
+}
+
+// Two CTAs per pair, four query tiles per pair; K is loaded in 64-key halves.
+cudaError_t launch_pair(const CUtensorMap& tq, const CUtensorMap& tk_half, const CUtensorMap& tv,
+                        const CUtensorMap& to, const FwdParams& p, cudaStream_t stream) {
+  dim3 grid(2 * ((p.n_q_tiles + 3) / 4), p.heads, p.batch);
+  ltx::ltx_attn_fwd_pair<<<grid, ltx::kPairThreads, ltx::PairSmem::kAlloc, stream>>>(
+      tq, tk_half, tv, to, p);
+  return cudaGetLastError();
+}
+
+// Launches the planned kernel (and, with key-range parts, the merge into `out`).  `tk_half`
+// is the key map with 64-row boxes, used by the pair kernel.
 cudaError_t launch_planned(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const CUtensorMap& to, const FwdParams& p, int head_dim, bool dual,
-                           int num_sms, void* out, cudaStream_t stream) {
+                           int num_sms, void* out, cudaStream_t stream,
+                           const CUtensorMap* tk_half = nullptr) {
   const bool split = p.num_splits > 1;
   cudaError_t e;
-  if (use_short_kv(p, num_sms)) {
+  if (tk_half && use_pair(p, head_dim, num_sms)) {
+    return launch_pair(tq, *tk_half, tv, to, p, stream);
+  } else if (use_short_kv(p, num_sms)) {
     return launch_skv(tq, tk, tv, to, p, head_dim, num_sms, stream);
   } else if (dual) {
     e = split ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
@@ -505,6 +527,9 @@ cudaError_t set_smem_limits_all() {
   if (e == cudaSuccess) e = set_smem_limits_skv();
   if (e == cudaSuccess) e = set_smem_limits_dual();
   if (e == cudaSuccess) e = set_smem_limits_na();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ltx::ltx_attn_fwd_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ltx::PairSmem::kAlloc);
   return e;
 }
 
@@ -572,11 +597,12 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
   if (splits_used) *splits_used = splits;
 
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv, to, tk_half;
   if (!encode_bshd(*c, &tq, q, q_len, batch, heads, head_dim) ||
       !encode_bshd(*c, &tk, k, kv_len, batch, heads, head_dim) ||
       !encode_bshd(*c, &tv, v, kv_len, batch, heads, head_dim) ||
-      !encode_bshd(*c, &to, out, q_len, batch, heads, head_dim))
+      !encode_bshd(*c, &to, out, q_len, batch, heads, head_dim) ||
+      !encode_bshd(*c, &tk_half, k, kv_len, batch, heads, head_dim, ltx::kBlockN / 2))
     return LTXATTN_ERR_CUDA;
 
   std::unique_lock<std::mutex> launch_lock(c->launch_mu, std::defer_lock);
@@ -610,7 +636,8 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
     if (cudaMemsetAsync(ws->ptr, 0xA5, need, stream) != cudaSuccess) return LTXATTN_ERR_CUDA;
 #endif
   }
-  cudaError_t e = launch_planned(tq, tk, tv, to, p, head_dim, dual, c->num_sms, out, stream);
+  cudaError_t e =
+      launch_planned(tq, tk, tv, to, p, head_dim, dual, c->num_sms, out, stream, &tk_half);
 #ifdef LTXATTN_DEBUG
   if (e == cudaSuccess && splits > 1) e = debug_check_guards(p, head_dim, stream);
 #endif

@@ -369,3 +369,29 @@ def test_two_host_threads_share_one_stream(oracle):
     for i, (q, k, v) in enumerate(cases):
         assert_parity(outs[i].cpu(), oracle.attention(q, k, v, 0.125, kv_valid_len=valids[i]),
                       f"thread case {i}")
+
+
+PAIR_SHAPES = [
+    # head_dim 128, at least 8 query tiles, unsplit: the CTA-pair kernel (cta_group::2).
+    # batch, heads, q_len, kv_len, kv_valid
+    (1, 1, 1024, 1024, 1024),    # two full pairs, one head
+    (2, 3, 1100, 1100, 1100),    # 9 query tiles: the last pair holds one real tile of four
+    (1, 2, 2048, 1000, 999),     # ragged last key tile (and a key side of 8 tiles)
+    (1, 2, 1280, 128, 77),       # one key tile, 77 valid keys (too few query tiles for the
+                                 # persistent short-key kernel)
+    (2, 2, 1536, 4096, 4000),    # many key tiles, masked tail
+]
+
+
+@pytest.mark.parametrize("shape", PAIR_SHAPES, ids=lambda s: "b{}h{}_q{}_kv{}v{}".format(*s))
+def test_cta_pair_kernel(oracle, shape):
+    b, h, lq, lkv, valid = shape
+    q, k, v = synth.make_qkv(b, lq, lkv, h, 128, seed=70 + lq + lkv, kv_valid=valid)
+    scale = 128 ** -0.5
+    got, used = gpu_run(q, k, v, valid, scale, num_splits=1)  # no key parts: the pair kernel
+    assert used == 1
+    rows = synth.sample_rows(b, lq, h, 48, seed=lq, full_heads=((b - 1, h - 1),))
+    i = torch.arange(lq - 100, lq)
+    rows = torch.unique(torch.cat([rows, (0 * lq + i) * h + 0]))
+    ref = oracle.attention(q, k, v, scale, kv_valid_len=valid, rows=rows.numpy())
+    assert_parity(got.reshape(-1, 128)[rows], ref, str(shape))
