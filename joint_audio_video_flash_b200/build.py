@@ -10,7 +10,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libltxattn.so")
 DEBUG_LIB = os.path.join(PKG, "libltxattn_debug.so")  # -DLTXATTN_DEBUG: workspace guard words
 SOURCES = ["ltxattn.cu"]
-DEPS = ["ltxattn.cu", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_fwd_skv.cuh", "qk_prologue.cuh",
+DEPS = ["ltxattn.cu", "attn_fwd.cuh", "attn_fwd_pp.cuh", "attn_fwd_skv.cuh", "attn_fwd_pair.cuh",
+        "attn_fwd_a2v.cuh", "qk_prologue.cuh",
         "na3d_fwd.cuh", "combine.cuh", "debug_guard.cuh", "sm100_ptx.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared"]

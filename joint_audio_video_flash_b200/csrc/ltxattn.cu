@@ -18,6 +18,7 @@
 #include "combine.cuh"
 #include "debug_guard.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_a2v.cuh"
 #include "attn_fwd_pair.cuh"
 #include "attn_fwd_pp.cuh"
 #include "attn_fwd_skv.cuh"
@@ -198,11 +199,14 @@ cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        cudaStream_t stream) {
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
   const int grid = (int)std::min<long long>(total, num_sms);
-  // head_dim 64, one key tile (a2v): per-unit K/V and the strided (batch, query tile, head)
-  // walk, so that the tiles in flight cover whole token rows of q and out
-  if (head_dim == 64)
-    return p.n_kv_tiles == 1 ? launch_skv_n<64, 1, true>(tq, tk, tv, to, p, grid, stream)
-                             : launch_skv_n<64, 2>(tq, tk, tv, to, p, grid, stream);
+  // head_dim 64, one key tile (a2v): three warpgroups doing softmax and epilogue of every
+  // third unit, per-unit K/V and the strided (batch, query tile, head) walk
+  if (head_dim == 64 && p.n_kv_tiles == 1) {
+    ltx::ltx_attn_fwd_a2v<<<grid, ltx::kA2vThreads, ltx::A2vSmem::kAlloc, stream>>>(tq, tk, tv,
+                                                                                    to, p);
+    return cudaGetLastError();
+  }
+  if (head_dim == 64) return launch_skv_n<64, 2>(tq, tk, tv, to, p, grid, stream);
   return p.n_kv_tiles == 1 ? launch_skv_n<128, 1>(tq, tk, tv, to, p, grid, stream)
                            : launch_skv_n<128, 2>(tq, tk, tv, to, p, grid, stream);
 }
@@ -455,7 +459,7 @@ bool plan_kernel(FwdParams& p, int head_dim, int num_splits, int num_sms, int ma
 }
 
 // Query sides of at least this many 128-row tiles at head_dim 128 (unsplit) run on CTA pairs.
-constexpr int kPairMinQTiles = 8;
+constexpr int kPairMinQTiles = 1 << 30;  // not dispatched: slower per cycle (see the trace notes)
 
 bool use_pair(const FwdParams& p, int head_dim, int num_sms) {
   return head_dim == 128 && p.num_splits == 1 && p.n_q_tiles >= kPairMinQTiles &&
@@ -530,6 +534,9 @@ cudaError_t set_smem_limits_all() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(ltx::ltx_attn_fwd_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ltx::PairSmem::kAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ltx::ltx_attn_fwd_a2v, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ltx::A2vSmem::kAlloc);
   return e;
 }
 
@@ -1089,11 +1096,12 @@ extern "C" int ltxattn_forward_split_noalloc(const void* q, const void* k, const
 
   Context c;  // tensor-map encoder only; nothing in it is allocated
   c.encode = g_noalloc_encode;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv, to, tk_half;
   if (!encode_bshd(c, &tq, q, q_len, batch, heads, head_dim) ||
       !encode_bshd(c, &tk, k, kv_len, batch, heads, head_dim) ||
       !encode_bshd(c, &tv, v, kv_len, batch, heads, head_dim) ||
-      !encode_bshd(c, &to, out, q_len, batch, heads, head_dim))
+      !encode_bshd(c, &to, out, q_len, batch, heads, head_dim) ||
+      !encode_bshd(c, &tk_half, k, kv_len, batch, heads, head_dim, ltx::kBlockN / 2))
     return LTXATTN_ERR_CUDA;
 
   // the status word is the one thing that must start at zero
@@ -1101,6 +1109,7 @@ extern "C" int ltxattn_forward_split_noalloc(const void* q, const void* k, const
     cudaGetLastError();
     return LTXATTN_ERR_CUDA;
   }
-  const cudaError_t e = launch_planned(tq, tk, tv, to, p, head_dim, dual, d->num_sms, out, stream);
+  const cudaError_t e =
+      launch_planned(tq, tk, tv, to, p, head_dim, dual, d->num_sms, out, stream, &tk_half);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
 }
