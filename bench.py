@@ -57,17 +57,47 @@ TRAFFIC = {
 }
 
 
-def kernel_label(c, num_sms: int = 148) -> str:
+def kernel_label(c, num_sms: int = 148, grouped: bool = False) -> str:
     """Name of the kernel the library's host dispatch picks for a call (report label only)."""
     qt = -(-c.q_len // 128)
     kt = -(-c.kv_valid_len // 128)
+    if c.head_dim == 64 and kt == 1 and (grouped or c.batch * c.heads * qt > num_sms):
+        return "ltx_attn_fwd_a2v (persistent, per-unit K/V" + (
+            ", grouped launch)" if grouped else ")")
     if kt <= 2 and c.batch * c.heads * qt > num_sms:
-        return f"ltx_attn_fwd_skv<{kt}> (persistent, K/V resident)"
+        return f"ltx_attn_fwd_skv<{c.head_dim}, {kt}> (persistent, K/V resident)"
     if c.head_dim == 64 and kt > 2 and qt <= 1:
         return "ltx_attn_fwd<64, 1 S buffer> (two CTAs per SM)"
     if qt >= 2:
         return f"ltx_attn_fwd_pp<{c.head_dim}> (two 128-row query tiles per CTA)"
     return f"ltx_attn_fwd<{c.head_dim}>"
+
+
+GROUP_MAX = 4  # calls per launch of the grouped kernel
+
+
+def launch_items(calls, grouped: bool = True):
+    """The step's API calls, as lists of indices into `calls`: the calls the library can
+    group (head_dim 64, every valid key in one 128-key tile: a2v and audio self-attention)
+    go together through forward_grouped when there are at least two; every other call is one
+    forward.  Order: each item where its first call stands."""
+    elig = [i for i, c in enumerate(calls) if c.head_dim == 64 and c.kv_valid_len <= 128]
+    if not grouped or len(elig) < 2:
+        return [[i] for i in range(len(calls))]
+    items = []
+    for i in range(len(calls)):
+        if i not in elig:
+            items.append([i])
+        elif i == elig[0]:
+            items.append(list(elig))
+    return items
+
+
+def item_launches(item, splits):
+    """Kernel launches of one launch item (a grouped item: one per GROUP_MAX calls)."""
+    if len(item) > 1:
+        return -(-len(item) // GROUP_MAX)
+    return 1 if splits[item[0]] == 1 else 2
 
 
 def kernel_source_hash(kernel: str = "video_self") -> str:
@@ -617,31 +647,41 @@ def run_ltxattn(args):
         dev_in.append(tuple(t.to(dev) for t in (q, k, v)))
         outs.append(torch.empty_like(dev_in[-1][0]))
 
+    items = launch_items(calls, grouped=not args.no_group)
+    splits = [1] * len(calls)
+
+    def launch(item):
+        if len(item) > 1:  # one forward_grouped: a2v and audio self-attention share a launch
+            ltxattn.forward_grouped([dict(q=dev_in[i][0], k=dev_in[i][1], v=dev_in[i][2],
+                                          out=outs[i], kv_valid_len=calls[i].kv_valid_len,
+                                          scale=calls[i].scale) for i in item])
+            return
+        i = item[0]
+        _, splits[i] = ltxattn.forward(*dev_in[i], outs[i], kv_valid_len=calls[i].kv_valid_len,
+                                       scale=calls[i].scale, return_splits=True)
+
     def step(events=None):
-        for i, c in enumerate(calls):
-            dq, dk, dv = dev_in[i]
+        for j, item in enumerate(items):
             if events is not None:
-                events[i][0].record(stream)
-            _, used = ltxattn.forward(dq, dk, dv, outs[i], kv_valid_len=c.kv_valid_len,
-                                      scale=c.scale, return_splits=True)
+                events[j][0].record(stream)
+            launch(item)
             if events is not None:
-                events[i][1].record(stream)
-            if len(splits) < len(calls):
-                splits.append(used)
+                events[j][1].record(stream)
 
     if args.once:  # one launch set, no timing: the command the Nsight Compute captures run
         step()
         torch.cuda.synchronize()
         ltxattn.check()
-        print(json.dumps({"workload": args.workload, "once": True, "splits": splits}))
+        print(json.dumps({"workload": args.workload, "once": True, "splits": splits,
+                          "items": items}))
         return
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize()
     ltxattn.check()
 
-    per_call = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in calls] for _ in range(args.steps)]
+    per_item = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in items] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     uuid = None
@@ -655,7 +695,7 @@ def run_ltxattn(args):
         wall0 = time.time()
         t_start.record(stream)
         for s in range(args.steps):
-            step(per_call[s])
+            step(per_item[s])
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -666,19 +706,52 @@ def run_ltxattn(args):
     step_flops = sum(c.flops for c in calls)
     value = whole_job_tflops(step_flops, args.steps, world, total_ms)
 
-    call_us, call_wall = [], []
-    for i, c in enumerate(calls):
-        ts = [per_call[s][i][0].elapsed_time(per_call[s][i][1]) * 1e3 for s in range(args.steps)]
-        call_us.append(ts)
-        call_wall.append([(wall0 + t_start.elapsed_time(per_call[s][i][0]) * 1e-3,
-                           wall0 + t_start.elapsed_time(per_call[s][i][1]) * 1e-3)
+    item_us, item_wall = [], []
+    for j in range(len(items)):
+        item_us.append([per_item[s][j][0].elapsed_time(per_item[s][j][1]) * 1e3
+                        for s in range(args.steps)])
+        item_wall.append([(wall0 + t_start.elapsed_time(per_item[s][j][0]) * 1e-3,
+                           wall0 + t_start.elapsed_time(per_item[s][j][1]) * 1e-3)
                           for s in range(args.steps)])
-    launches_per_step = sum(1 if sp == 1 else 2 for sp in splits)
+    launches_per_step = sum(item_launches(it, splits) for it in items)
+
+    # ---- the members of a grouped launch, timed once more (outside the timed region, L2
+    # flushed before every call, interleaved so that all see the same clocks): the whole
+    # group, each member alone through forward (its own launch and kernel), and the group
+    # without it through forward_grouped, so that the group's time splits into what each
+    # member adds to the shared launch
+    item_of = {i: j for j, it in enumerate(items) for i in it}
+    member_us = {}
+    groups = [it for it in items if len(it) > 1]
+    if groups:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        fns, keys = [], []
+        for gi, it in enumerate(groups):
+            fns.append(lambda it=it: launch(it))
+            keys.append(("group", gi))
+            for i in it:
+                fns.append(lambda i=i: ltxattn.forward(*dev_in[i], outs[i],
+                                                       kv_valid_len=calls[i].kv_valid_len,
+                                                       scale=calls[i].scale))
+                keys.append(("alone", i))
+                rest = [x for x in it if x != i]
+                fns.append(lambda rest=rest: launch(rest) if len(rest) > 1 else
+                           ltxattn.forward_grouped([dict(
+                               q=dev_in[rest[0]][0], k=dev_in[rest[0]][1], v=dev_in[rest[0]][2],
+                               out=outs[rest[0]], kv_valid_len=calls[rest[0]].kv_valid_len,
+                               scale=calls[rest[0]].scale)]))
+                keys.append(("without", i))
+        us_m, _ = timed_calls(fns, args.steps, 3, stream, flush)
+        ltxattn.check()
+        member_us = dict(zip(keys, us_m))
+        del flush
+        step()  # outs hold the timed configuration's results again (checked below)
+        torch.cuda.synchronize()
 
     # ---- end to end through the public API with host buffers.  Every step uploads all
     # inputs from pinned host memory and downloads every output; uploads run on one copy
-    # stream and downloads on another (PCIe is full duplex), each call's kernel waits for
-    # its own upload, and an upload into a device buffer waits for the previous step's
+    # stream and downloads on another (PCIe is full duplex), each launch item waits for
+    # its own uploads, and an upload into a device buffer waits for the previous step's
     # kernel that read it.
     pinned = [tuple(t.pin_memory() for t in trip) for trip in host]
     host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
@@ -687,34 +760,35 @@ def run_ltxattn(args):
     e2e_steps = max(1, min(args.steps, 5))
     up_stream = torch.cuda.Stream(device=dev)
     down_stream = torch.cuda.Stream(device=dev)
-    consumed = [None] * len(calls)   # event: call i's kernel of the previous step finished
-    drained = [None] * len(calls)    # event: call i's output of the previous step downloaded
+    consumed = [None] * len(items)  # event: item j's kernels of the previous step finished
+    drained = [None] * len(calls)   # event: call i's output of the previous step downloaded
 
     def e2e_step():
-        for i, c in enumerate(calls):
-            dq, dk, dv = dev_in[i]
-            hq, hk, hv = pinned[i]
+        for j, item in enumerate(items):
             with torch.cuda.stream(up_stream):
-                if consumed[i] is not None:
-                    up_stream.wait_event(consumed[i])
-                dq.copy_(hq, non_blocking=True)
-                dk.copy_(hk, non_blocking=True)
-                dv.copy_(hv, non_blocking=True)
+                if consumed[j] is not None:
+                    up_stream.wait_event(consumed[j])
+                for i in item:
+                    for d_t, h_t in zip(dev_in[i], pinned[i]):
+                        d_t.copy_(h_t, non_blocking=True)
                 uploaded = torch.cuda.Event()
                 uploaded.record(up_stream)
             stream.wait_event(uploaded)
-            if drained[i] is not None:
-                stream.wait_event(drained[i])
-            ltxattn.forward(dq, dk, dv, outs[i], kv_valid_len=c.kv_valid_len, scale=c.scale)
+            for i in item:
+                if drained[i] is not None:
+                    stream.wait_event(drained[i])
+            launch(item)
             done = torch.cuda.Event()
             done.record(stream)
-            consumed[i] = done
+            consumed[j] = done
             with torch.cuda.stream(down_stream):
                 down_stream.wait_event(done)
-                host_out[i].copy_(outs[i], non_blocking=True)
+                for i in item:
+                    host_out[i].copy_(outs[i], non_blocking=True)
                 ev = torch.cuda.Event()
                 ev.record(down_stream)
-                drained[i] = ev
+                for i in item:
+                    drained[i] = ev
 
     e2e_step()
     torch.cuda.synchronize()
@@ -743,7 +817,8 @@ def run_ltxattn(args):
     # region (the sustained figure was measured at the power-capped clock), else the
     # sustained one.
     vi = max(range(len(calls)), key=lambda i: calls[i].flops)
-    v_us = statistics.mean(call_us[vi])
+    assert items[item_of[vi]] == [vi], "the dominant call runs on its own launch"
+    v_us = statistics.mean(item_us[item_of[vi]])
     clk = clocks.summary()
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -773,21 +848,32 @@ def run_ltxattn(args):
 
     per_call_out = {}
     for i, c in enumerate(calls):
-        us = statistics.median(call_us[i])
-        tfl = c.flops / (us * 1e-6) / 1e12
-        gbs = c.bytes / (us * 1e-6) / 1e9
-        per_call_out[c.name] = {
-            "us_median": us, "us_p10": sorted(call_us[i])[max(0, int(0.1 * len(call_us[i])))],
-            "us_p90": sorted(call_us[i])[min(len(call_us[i]) - 1, int(0.9 * len(call_us[i])))],
-            "tflops": tfl, "frac_bf16_peak": tfl / float(peaks.get("bf16_tflops", 1590.0)),
-            "gbs": gbs, "frac_hbm": gbs / float(peaks.get("hbm_gbs", 6650.0)),
+        j = item_of[i]
+        grouped = len(items[j]) > 1
+        us_list = member_us[("alone", i)] if grouped else item_us[j]
+        entry = dist_stats(us_list)
+        entry.update(call_roofline(c.flops, c.bytes, entry["us_median"], peaks))
+        entry.update({
             "shape": f"B{c.batch} Lq{c.q_len} Lkv{c.kv_len} valid{c.kv_valid_len} "
                      f"H{c.heads} D{c.head_dim}",
-            "splits": splits[i], "kernel": kernel_label(c)}
+            "splits": splits[i], "kernel": kernel_label(c)})
+        if grouped:  # us_* above: the call alone (its own launch), timed after the step
+            group_alone = statistics.median(member_us[("group", groups.index(items[j]))])
+            without = statistics.median(member_us[("without", i)])
+            entry["timed_alone"] = True
+            entry["group"] = {
+                "members": [calls[x].name for x in items[j]],
+                "kernel": kernel_label(c, grouped=True),
+                "us_median_in_step": statistics.median(item_us[j]),  # the timed step
+                # the next three from the interleaved loop after the step (L2 flushed)
+                "us_median": group_alone,
+                "us_without_this_call": without,
+                "us_added_by_this_call": group_alone - without}
         if c.flops / c.bytes > 1000:  # tensor-bound: time beside the SM clock it ran at
-            per_call_out[c.name]["clock"] = clock_normalised(call_us[i], call_wall[i], trace)
+            entry["clock"] = clock_normalised(item_us[j], item_wall[j], trace)
         if rank == 0 and not args.no_parity:  # the oracle on sampled rows, after the timing
-            per_call_out[c.name]["parity"] = attention_parity(c, *host[i], outs[i], seed=c.seed)
+            entry["parity"] = attention_parity(c, *host[i], outs[i], seed=c.seed)
+        per_call_out[c.name] = entry
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -803,6 +889,7 @@ def run_ltxattn(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "per_call": per_call_out,
+        "launch_items": [[calls[i].name for i in it] for it in items],
     }
     if rank == 0 and world == 1 and not args.no_per_config and args.workload == "block768":
         del dev_in, pinned
@@ -1373,6 +1460,9 @@ def main():
     ap.add_argument("--no-parity", action="store_true",
                     help="skip the oracle comparison of the timed outputs")
     ap.add_argument("--per-config-steps", type=int, default=10)
+    ap.add_argument("--no-group", action="store_true",
+                    help="launch a2v and audio self-attention separately (forward per call) "
+                         "instead of through one forward_grouped")
     ap.add_argument("--once", action="store_true",
                     help="run each call of the workload once and exit (profiling)")
     ap.add_argument("--cp", action="store_true",

@@ -129,6 +129,48 @@ LTXATTN_API int ltxattn_forward_ex(const void* q, const void* k, const void* v, 
                        int kv_len, int kv_valid_len, int batch, int heads, int head_dim,
                        float scale, int num_splits, int* splits_used, ltxattn_stream_t stream);
 
+/* One call of ltxattn_forward_grouped: the arguments of ltxattn_forward of the same names. */
+typedef struct ltxattn_call {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  int q_len;
+  int kv_len;
+  int kv_valid_len;
+  int batch;
+  int heads;
+  int head_dim;
+  float scale;
+} ltxattn_call;
+
+/* Most calls one ltxattn_forward_grouped takes (more give LTXATTN_ERR_UNSUPPORTED). */
+#define LTXATTN_MAX_GROUP 64
+
+/*
+ * Several independent attention calls in as few launches as possible.  An LTX-2 block runs
+ * four attentions per step ("LTX-2: replicate audio stream across Ulysses ranks by
+ * default", Description): two of them, a2v (video queries over the audio keys) and audio
+ * self-attention, have every valid key in one 128-key tile at head_dim 64, and audio
+ * self-attention is so small (one query tile per head) that its own launch costs more than
+ * its work.  Here such calls (head_dim 64, kv_valid_len <= 128) share one persistent launch,
+ * up to four per launch, their (batch, query tile, head) units walked as one sequence by all
+ * SMs; every other call runs as ltxattn_forward runs it, in the order given.
+ *
+ *   calls    host array of n_calls descriptors (read during the call only; the pointers in
+ *            it are device pointers, as for ltxattn_forward)
+ *   n_calls  1 .. LTXATTN_MAX_GROUP
+ * Each call computes what ltxattn_forward computes (same arithmetic and precision; a grouped
+ * call may run on another kernel than the same call alone, so results agree to rounding,
+ * not bit for bit).  Every call is checked as ltxattn_forward checks it, and no call's `out`
+ * may overlap another call's q, k, v or out (INVALID_ARG); all checks run before anything
+ * is enqueued.  Needs ltxattn_create.  Asynchronous on `stream`; LTXATTN_ERR_CUDA on a
+ * failed launch (calls before it stay enqueued); a kernel wait that times out is reported by
+ * ltxattn_check.
+ */
+LTXATTN_API int ltxattn_forward_grouped(const ltxattn_call* calls, int n_calls,
+                                        ltxattn_stream_t stream);
+
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device (LTXATTN_ERR_WORKSPACE_GUARD for a guard error in the debug

@@ -1,23 +1,23 @@
 // attn_fwd_skv.cuh -- attention forward for a short key side (at most 256 keys) on
-// sm_100a: a2v (video queries over the padded audio keys/values) of an LTX-2 block
-// ("LTX-2: replicate audio stream across Ulysses ranks by default", Description), at
-// head_dim 64, and the streams' queries over a padded text context at head_dim 64 or
-// 128.  Same operation, layout and key mask as
-// attn_fwd.cuh.  With every key in one S tile the softmax max is exact, so there is
-// no online rescale.  The work is bound by HBM (reading Q, writing O) and by the
-// exponentials, so the design keeps both busy at once:
+// sm_100a: the streams' queries over a padded text context at head_dim 64 or 128, and a2v
+// (video queries over the padded audio keys/values of an LTX-2 block, "LTX-2: replicate
+// audio stream across Ulysses ranks by default", Description) when the audio side has more
+// than 128 valid keys.  (With at most 128 valid keys at head_dim 64, a2v runs on
+// attn_fwd_a2v.cuh.)  Same operation, layout and key mask as attn_fwd.cuh.  With every key
+// in one S tile the softmax max is exact, so there is no online rescale.  The work is bound
+// by HBM (reading Q, writing O) and by the exponentials, so the design keeps both busy at
+// once:
 //
 //   - persistent: one CTA per SM walks a contiguous run of query tiles (flattened
 //     over batch, head, tile); K and V of the current (batch, head) stay resident in
 //     shared memory and are reloaded only when the run crosses into the next head;
-//   - warp 0 streams Q tiles through a deep TMA ring (8 stages for one key tile);
+//   - warp 0 streams Q tiles through a deep TMA ring;
 //   - warp 1 issues S = Q K^T two tiles ahead of O = P V, so a softmax warpgroup
 //     finds its next scores computed when it finishes a tile;
 //   - warps 4-11: two softmax warpgroups take alternate tiles (S -> P and the row
 //     sum l); they never wait for the PV product;
 //   - warps 12-15: the epilogue warpgroup takes every tile in order: waits for O,
-//     divides by l, rounds to bf16, stages the tile (two staging buffers) and
-//     issues its TMA store.
+//     divides by l, rounds to bf16, stages the tile and issues its TMA store.
 // TMEM (512 columns) holds NB buffers (4 / NKV at head_dim 64, 2 at 128); tile i uses
 // buffer i % NB.  In a buffer: S over the first 128*NKV columns, P packed as bf16 pairs
 // over the first 64*NKV columns (written after the scores it replaces were read), O (D
@@ -41,26 +41,17 @@ static_assert(128 * kSkvRegsIssue + 128 * kSkvRegsEpi + 256 * kSkvRegsSoftmax <=
                   kSkvThreads * kSkvRegsLaunch,
               "register split exceeds the launch allocation");
 
-// kTileKV = false: K/V of the current (batch, head) stay resident (reloaded when the
-// CTA's contiguous run of units crosses into the next head); Q streams through a ring.
-// kTileKV = true (head_dim 64, one key tile): every unit brings its own K and V (a few
-// KB, L2-resident for all heads) with its Q, and CTA c takes units c, c + G, c + 2G, ...
-// (G = the grid) of the order (batch, query tile, head), head fastest: the G tiles loaded
-// at once are then every head of a few token blocks, i.e. whole contiguous token rows of
-// q and out, instead of 128-byte rows 4 KB apart of unrelated heads and token blocks.
-// Q and K share a ring of stages (freed once QK has read them), V has its own (freed by PV).
-template <int D, int NKV, bool kTileKV = false>
+// K/V of the current (batch, head) stay resident (reloaded when the CTA's contiguous run
+// of units crosses into the next head); Q streams through a ring.
+template <int D, int NKV>
 struct SkvSmem {
   static_assert(NKV == 1 || NKV == 2, "one or two 128-key tiles");
   static_assert(D == 64 || D == 128, "head_dim");
-  static_assert(!kTileKV || (D == 64 && NKV == 1), "per-tile K/V: head_dim 64, one key tile");
   static constexpr int kBoxes = D / 64;            // 64-column (128-byte) boxes per row
   static constexpr int kBoxBytes = kBlockM * 128;  // 128 rows x 64 bf16
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kQStages =
-      kTileKV ? 4 : D == 64 ? (NKV == 1 ? 8 : 6) : (NKV == 1 ? 3 : 2);
-  static constexpr int kVStages = kTileKV ? 4 : 1;       // V ring (per-tile K/V only)
-  static constexpr int kStaging = kTileKV ? 1 : D == 64 ? 2 : 1;  // output staging tiles
+  static constexpr int kQStages = D == 64 ? (NKV == 1 ? 8 : 6) : (NKV == 1 ? 3 : 2);
+  static constexpr int kStaging = D == 64 ? 2 : 1;     // output staging tiles
   static constexpr uint32_t kBufCols = D == 64 ? 128u * NKV : 256u;  // columns per buffer
   static constexpr int kNB = (int)(512u / kBufCols);    // TMEM buffers
   // QK runs this many tiles ahead of PV; QK(i + kLookahead) reuses the buffer of tile
@@ -68,14 +59,11 @@ struct SkvSmem {
   static constexpr int kLookahead = kNB - 1 < 2 ? kNB - 1 : 2;
   static constexpr uint32_t kColO = 64u * NKV;          // O within a buffer (after P)
   static_assert(kColO + D <= kBufCols, "O fits its buffer");
-  // resident K/V: K [box][key tile], V, then the Q ring; per-tile K/V: stage s of the QK
-  // ring holds Q then K, then the V ring
-  static constexpr int kQKStride = kTileKV ? 2 * kTileBytes : kTileBytes;  // Q ring stride
-  static constexpr int kK = kTileKV ? kTileBytes : 0;   // K of stage 0 (per-tile: after Q)
-  static constexpr int kQ = kTileKV ? 0 : 2 * NKV * kTileBytes;  // Q ring
-  static constexpr int kV = kTileKV ? kQStages * kQKStride : NKV * kTileBytes;
-  static constexpr int kStage =                                  // output staging
-      kTileKV ? kV + kVStages * kTileBytes : kQ + kQStages * kTileBytes;
+  // K [box][key tile], V, then the Q ring
+  static constexpr int kK = 0;
+  static constexpr int kV = NKV * kTileBytes;
+  static constexpr int kQ = 2 * NKV * kTileBytes;
+  static constexpr int kStage = kQ + kQStages * kTileBytes;  // output staging
   static constexpr int kRowSum = kStage + kStaging * kTileBytes;  // l per buffer and row
   static constexpr int kBar = kRowSum + kNB * kBlockM * 4;
   static constexpr int bKVF = 0;
@@ -86,9 +74,7 @@ struct SkvSmem {
   static constexpr int bPF = bSF + kNB;         // kNB
   static constexpr int bOF = bPF + kNB;         // kNB
   static constexpr int bTF = bOF + kNB;         // kNB: TMEM buffer free
-  static constexpr int bVF = bTF + kNB;         // kVStages (per-tile K/V)
-  static constexpr int bVE = bVF + kVStages;    // kVStages
-  static constexpr int bDrain = bVE + kVStages;
+  static constexpr int bDrain = bTF + kNB;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
@@ -100,17 +86,6 @@ struct SkvSmem {
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
   static_assert(kLookahead >= 1 && kLookahead <= kNB - 1 && kLookahead < kQStages,
                 "pipeline depth");
-};
-
-// Unit u of the per-tile K/V walk: order (batch, query tile, head), head fastest.
-struct SkvUnit {
-  int b, h, qt;
-  __device__ __forceinline__ void init(long long u, const FwdParams& p) {
-    const long long t = u / p.heads;
-    h = (int)(u - t * p.heads);
-    b = (int)(t / p.n_q_tiles);
-    qt = (int)(t - (long long)b * p.n_q_tiles);
-  }
 };
 
 // (batch, head, query tile) of consecutive flattened tile indices, advanced without
@@ -135,13 +110,13 @@ struct SkvCursor {
   }
 };
 
-template <int D, int NKV, bool kTileKV = false>
+template <int D, int NKV>
 __global__ void __launch_bounds__(kSkvThreads, 1)
     ltx_attn_fwd_skv(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
-  using L = SkvSmem<D, NKV, kTileKV>;
+  using L = SkvSmem<D, NKV>;
   constexpr int NB = L::kNB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -154,14 +129,11 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // resident K/V: a contiguous run of flattened (batch, head, query tile) indices for this
-  // CTA; per-tile K/V: units blockIdx.x + i * gridDim.x of the (batch, query tile, head) order
+  // a contiguous run of flattened (batch, head, query tile) indices for this CTA
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
-  const long long t_begin = kTileKV ? 0 : total * blockIdx.x / gridDim.x;
+  const long long t_begin = total * blockIdx.x / gridDim.x;
   const long long t_end = total * (blockIdx.x + 1) / gridDim.x;
-  const int cnt = kTileKV ? (int)((total - blockIdx.x + gridDim.x - 1) / gridDim.x)
-                          : (int)(t_end - t_begin);
-  auto unit_of = [&](int i) -> long long { return (long long)blockIdx.x + (long long)i * gridDim.x; };
+  const int cnt = (int)(t_end - t_begin);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::bKVF), 1);
@@ -169,10 +141,6 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
     for (int s = 0; s < L::kQStages; ++s) {
       mbar_init(bar(L::bQF + s), 1);
       mbar_init(bar(L::bQE + s), 1);
-    }
-    for (int s = 0; s < L::kVStages; ++s) {
-      mbar_init(bar(L::bVF + s), 1);
-      mbar_init(bar(L::bVE + s), 1);
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(bar(L::bSF + b), 1);
@@ -199,44 +167,7 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     setmaxnreg_dec<kSkvRegsIssue>();
-    if (kTileKV && lane == 0 && !*abort_flag && cnt > 0) {
-      // every unit: Q and K into a stage of the QK ring, V into the V ring
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      int last_q[L::kQStages], last_v[L::kVStages];
-      for (int s = 0; s < L::kQStages; ++s) last_q[s] = -1;
-      for (int s = 0; s < L::kVStages; ++s) last_v[s] = -1;
-      bool ok = true;
-      for (int i = 0; i < cnt && ok; ++i) {
-        SkvUnit u;
-        u.init(unit_of(i), p);
-        const int qs = i % L::kQStages;
-        ok = mbar_wait_lean(bar(L::bQE + qs), ((uint32_t)(i / L::kQStages) & 1u) ^ 1u, ctl);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::bQF + qs), 2 * L::kTileBytes);
-        tma_load_4d(sbase + L::kQ + qs * L::kQKStride, &tm_q, bar(L::bQF + qs), 0, u.h,
-                    u.qt * kBlockM, u.b);
-        tma_load_4d(sbase + L::kK + qs * L::kQKStride, &tm_k, bar(L::bQF + qs), 0, u.h, 0, u.b);
-        last_q[qs] = i;
-        const int vs = i % L::kVStages;
-        ok = mbar_wait_lean(bar(L::bVE + vs), ((uint32_t)(i / L::kVStages) & 1u) ^ 1u, ctl);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::bVF + vs), L::kTileBytes);
-        tma_load_4d(sbase + L::kV + vs * L::kTileBytes, &tm_v, bar(L::bVF + vs), 0, u.h, 0, u.b);
-        last_v[vs] = i;
-      }
-      if (!ok) {
-        for (int s = 0; s < L::kQStages; ++s)
-          if (last_q[s] >= 0)
-            mbar_wait_drain(bar(L::bQF + s), (uint32_t)(last_q[s] / L::kQStages) & 1u,
-                            p.timeout_ns);
-        for (int s = 0; s < L::kVStages; ++s)
-          if (last_v[s] >= 0)
-            mbar_wait_drain(bar(L::bVF + s), (uint32_t)(last_v[s] / L::kVStages) & 1u,
-                            p.timeout_ns);
-      }
-    } else if (!kTileKV && lane == 0 && !*abort_flag && cnt > 0) {
+    if (lane == 0 && !*abort_flag && cnt > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -315,8 +246,8 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
             !wt(bar(L::bTF + bf), ((uint32_t)(i / NB) & 1u) ^ 1u))
           return false;
         tc_fence_after();
-        const uint32_t q_off = (uint32_t)qs * L::kQKStride;
-        const uint32_t k_off = kTileKV ? q_off : 0u;  // per-tile K sits beside its Q
+        const uint32_t q_off = (uint32_t)qs * L::kTileBytes;
+        const uint32_t k_off = 0u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // 16 head-dim columns: box kk / 4, 32-byte step kk % 4 within the box
@@ -333,18 +264,15 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       // O = P_i V into buffer i % NB (waits for P_i)
       auto pv = [&](int i) -> bool {
         const int bf = i % NB;
-        const int vs = i % L::kVStages;
         if (!wt(bar(L::bPF + bf), (uint32_t)(i / NB) & 1u)) return false;
-        if (kTileKV && !wt(bar(L::bVF + vs), (uint32_t)(i / L::kVStages) & 1u)) return false;
         tc_fence_after();
         const uint32_t buf = tmem + L::kBufCols * bf;
-        const uint32_t v_off = kTileKV ? (uint32_t)vs * L::kTileBytes : 0u;
+        const uint32_t v_off = 0u;
 #pragma unroll
         for (int kk = 0; kk < (kBlockN / 16) * NKV; ++kk)
           umma_ts_elect(buf + L::kColO, buf + kk * 8, dv.at(v_off + kk * 16 * 128), idesc_pv,
                         kk > 0 ? 1u : 0u);
         umma_commit_elect(bar(L::bOF + bf));
-        if (kTileKV) umma_commit_elect(bar(L::bVE + vs));  // this V stage may be refilled
         return true;
       };
       // QK runs up to kLookahead tiles ahead of PV but never into the next (batch, head)
@@ -355,16 +283,11 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       bool q_fresh = true;    // tile nq starts a (batch, head)
       bool ok = true;
       for (int i = 0; i < cnt && ok; ++i) {
-        if constexpr (kTileKV) {
-          // every unit has its own K/V: QK simply runs kLookahead units ahead of PV
-          while (ok && nq < cnt && nq <= i + L::kLookahead) ok = qk(nq++, false);
-        } else {
-          while (ok && nq < cnt && nq <= i + L::kLookahead && (!q_fresh || nq == i)) {
-            if (q_fresh && nq > 0) umma_commit_elect(bar(L::bKVE));  // old K/V may be overwritten
-            ok = qk(nq, q_fresh);
-            ++nq;
-            q_fresh = cq.advance(p);
-          }
+        while (ok && nq < cnt && nq <= i + L::kLookahead && (!q_fresh || nq == i)) {
+          if (q_fresh && nq > 0) umma_commit_elect(bar(L::bKVE));  // old K/V may be overwritten
+          ok = qk(nq, q_fresh);
+          ++nq;
+          q_fresh = cq.advance(p);
         }
         if (ok) ok = pv(i);
       }
@@ -527,18 +450,10 @@ __global__ void __launch_bounds__(kSkvThreads, 1)
       fence_proxy_async_smem();
       named_bar_sync(1, kBlockM);
       if (leader) {
-        int sh = cur.h, sqt = cur.qt, sbat = cur.b;
-        if constexpr (kTileKV) {
-          SkvUnit u;
-          u.init(unit_of(i), p);
-          sh = u.h;
-          sqt = u.qt;
-          sbat = u.b;
-        }
 #pragma unroll
         for (int bx = 0; bx < L::kBoxes; ++bx)
           tma_store_4d(&tm_o, sbase + L::kStage + sb * L::kTileBytes + bx * L::kBoxBytes,
-                       bx * 64, sh, sqt * kBlockM, sbat);
+                       bx * 64, cur.h, cur.qt * kBlockM, cur.b);
         tma_store_commit();
       }
       cur.advance(p);

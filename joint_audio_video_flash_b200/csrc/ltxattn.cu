@@ -65,7 +65,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_check",         "ltxattn_destroy",          "ltxattn_status_string",
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
     "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope", "ltxattn_na3d_forward",
-    "ltxattn_forward_partial", "ltxattn_combine",
+    "ltxattn_forward_partial", "ltxattn_combine", "ltxattn_forward_grouped",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -184,14 +184,47 @@ bool use_short_kv(const FwdParams& p, int num_sms) {
          (long long)p.batch * p.heads * p.n_q_tiles > num_sms;
 }
 
-template <int D, int NKV, bool kTileKV = false>
+template <int D, int NKV>
 cudaError_t launch_skv_n(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& to, const FwdParams& p, int grid,
                          cudaStream_t stream) {
-  ltx::ltx_attn_fwd_skv<D, NKV, kTileKV>
-      <<<grid, ltx::kSkvThreads, ltx::SkvSmem<D, NKV, kTileKV>::kAlloc, stream>>>(tq, tk, tv,
+  ltx::ltx_attn_fwd_skv<D, NKV>
+      <<<grid, ltx::kSkvThreads, ltx::SkvSmem<D, NKV>::kAlloc, stream>>>(tq, tk, tv,
                                                                                  to, p);
   return cudaGetLastError();
+}
+
+// Appends a call (its maps and sizes) to a group of the a2v kernel.
+void a2v_append(ltx::A2vArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                const CUtensorMap& tv, const CUtensorMap& to, const FwdParams& p) {
+  const int j = a.n_problems++;
+  a.q[j] = tq;
+  a.k[j] = tk;
+  a.v[j] = tv;
+  a.o[j] = to;
+  ltx::A2vProblem& pr = a.prob[j];
+  pr.batch = p.batch;
+  pr.heads = p.heads;
+  pr.n_q_tiles = p.n_q_tiles;
+  pr.kv_valid = p.kv_valid;
+  pr.scale_log2 = p.scale_log2;
+  pr.first_unit = a.total_units;
+  a.total_units += (long long)p.batch * p.heads * p.n_q_tiles;
+  a.status = p.status;
+  a.timeout_ns = p.timeout_ns;
+}
+
+// One persistent CTA per SM (fewer with fewer units) over every unit of the group.
+cudaError_t launch_a2v(const ltx::A2vArgs& a, int num_sms, cudaStream_t stream) {
+  const int grid = (int)std::min<long long>(a.total_units, num_sms);
+  ltx::ltx_attn_fwd_a2v<<<grid, ltx::kA2vThreads, ltx::A2vSmem::kAlloc, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// Calls the a2v kernel takes (alone or grouped): head_dim 64, every valid key in one tile,
+// no key split.
+bool a2v_eligible(const FwdParams& p, int head_dim) {
+  return head_dim == 64 && p.n_kv_tiles == 1 && p.num_splits == 1;
 }
 
 cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -201,10 +234,10 @@ cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const int grid = (int)std::min<long long>(total, num_sms);
   // head_dim 64, one key tile (a2v): three warpgroups doing softmax and epilogue of every
   // third unit, per-unit K/V and the strided (batch, query tile, head) walk
-  if (head_dim == 64 && p.n_kv_tiles == 1) {
-    ltx::ltx_attn_fwd_a2v<<<grid, ltx::kA2vThreads, ltx::A2vSmem::kAlloc, stream>>>(tq, tk, tv,
-                                                                                    to, p);
-    return cudaGetLastError();
+  if (a2v_eligible(p, head_dim)) {
+    ltx::A2vArgs a{};
+    a2v_append(a, tq, tk, tv, to, p);
+    return launch_a2v(a, num_sms, stream);
   }
   if (head_dim == 64) return launch_skv_n<64, 2>(tq, tk, tv, to, p, grid, stream);
   return p.n_kv_tiles == 1 ? launch_skv_n<128, 1>(tq, tk, tv, to, p, grid, stream)
@@ -251,17 +284,15 @@ cudaError_t set_smem_limits_pp() {
                               ltx::PPSmem<D>::kAlloc);
 }
 
-template <int D, int NKV, bool kTileKV = false>
+template <int D, int NKV>
 cudaError_t set_smem_limit_skv() {
-  return cudaFuncSetAttribute(ltx::ltx_attn_fwd_skv<D, NKV, kTileKV>,
+  return cudaFuncSetAttribute(ltx::ltx_attn_fwd_skv<D, NKV>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              ltx::SkvSmem<D, NKV, kTileKV>::kAlloc);
+                              ltx::SkvSmem<D, NKV>::kAlloc);
 }
 
 cudaError_t set_smem_limits_skv() {
-  cudaError_t e = set_smem_limit_skv<64, 1>();
-  if (e == cudaSuccess) e = set_smem_limit_skv<64, 1, true>();
-  if (e == cudaSuccess) e = set_smem_limit_skv<64, 2>();
+  cudaError_t e = set_smem_limit_skv<64, 2>();
   if (e == cudaSuccess) e = set_smem_limit_skv<128, 1>();
   if (e == cudaSuccess) e = set_smem_limit_skv<128, 2>();
   return e;
@@ -540,53 +571,9 @@ cudaError_t set_smem_limits_all() {
   return e;
 }
 
-}  // namespace
-
-extern "C" {
-
-int ltxattn_create(void) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
-    cudaGetLastError();
-    return LTXATTN_ERR_CUDA;
-  }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_ctx.count(dev)) return LTXATTN_OK;
-  Context* c = new Context();
-  c->device = dev;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  bool ok = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) ==
-                cudaSuccess &&
-            cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess && fn != nullptr;
-  if (ok) {
-    c->encode = reinterpret_cast<EncodeTiledFn>(fn);
-    ok = cudaMalloc(&c->d_status, sizeof(int)) == cudaSuccess &&
-         cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
-         set_smem_limits_all() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
-  }
-  if (!ok) {
-    cudaGetLastError();
-    if (c->d_status) cudaFree(c->d_status);
-    delete c;
-    return LTXATTN_ERR_CUDA;
-  }
-  g_ctx[dev] = c;
-  return LTXATTN_OK;
-}
-
-int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, int q_len,
-                       int kv_len, int kv_valid_len, int batch, int heads, int head_dim,
-                       float scale, int num_splits, int* splits_used, ltxattn_stream_t stream_) {
-  int st = validate(q, k, v, out, q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale);
-  if (st != LTXATTN_OK) return st;
-  if (num_splits < 0) return LTXATTN_ERR_INVALID_ARG;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  Context* c = current_context(&st);
-  if (!c) return st;
-
+// FwdParams of a validated call, before planning.
+FwdParams call_params(const Context& c, int q_len, int kv_len, int kv_valid_len, int batch,
+                      int heads, float scale) {
   FwdParams p{};
   p.q_len = q_len;
   p.kv_len = kv_len;
@@ -596,9 +583,17 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   p.n_q_tiles = (q_len + ltx::kBlockM - 1) / ltx::kBlockM;
   p.n_kv_tiles = (kv_valid_len + ltx::kBlockN - 1) / ltx::kBlockN;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.status = c->d_status;
+  p.status = c.d_status;
   p.timeout_ns = kDefaultTimeoutNs;
+  return p;
+}
 
+// One validated call on context `c`: plans it (num_splits as ltxattn_forward_ex takes it),
+// takes the stream's workspace for key-range partials and enqueues the kernels.
+int forward_one(Context* c, const void* q, const void* k, const void* v, void* out, int q_len,
+                int kv_len, int kv_valid_len, int batch, int heads, int head_dim, float scale,
+                int num_splits, int* splits_used, cudaStream_t stream) {
+  FwdParams p = call_params(*c, q_len, kv_len, kv_valid_len, batch, heads, scale);
   const bool dual = plan_kernel(p, head_dim, num_splits, c->num_sms, 0);
   const int splits = p.num_splits;
   if ((long long)batch * splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
@@ -649,6 +644,110 @@ int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, i
   if (e == cudaSuccess && splits > 1) e = debug_check_guards(p, head_dim, stream);
 #endif
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ltxattn_create(void) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return LTXATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_ctx.count(dev)) return LTXATTN_OK;
+  Context* c = new Context();
+  c->device = dev;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  bool ok = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev) ==
+                cudaSuccess &&
+            cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && fn != nullptr;
+  if (ok) {
+    c->encode = reinterpret_cast<EncodeTiledFn>(fn);
+    ok = cudaMalloc(&c->d_status, sizeof(int)) == cudaSuccess &&
+         cudaMemset(c->d_status, 0, sizeof(int)) == cudaSuccess &&
+         set_smem_limits_all() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
+  }
+  if (!ok) {
+    cudaGetLastError();
+    if (c->d_status) cudaFree(c->d_status);
+    delete c;
+    return LTXATTN_ERR_CUDA;
+  }
+  g_ctx[dev] = c;
+  return LTXATTN_OK;
+}
+
+int ltxattn_forward_ex(const void* q, const void* k, const void* v, void* out, int q_len,
+                       int kv_len, int kv_valid_len, int batch, int heads, int head_dim,
+                       float scale, int num_splits, int* splits_used, ltxattn_stream_t stream_) {
+  int st = validate(q, k, v, out, q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale);
+  if (st != LTXATTN_OK) return st;
+  if (num_splits < 0) return LTXATTN_ERR_INVALID_ARG;
+  Context* c = current_context(&st);
+  if (!c) return st;
+  return forward_one(c, q, k, v, out, q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale,
+                     num_splits, splits_used, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+int ltxattn_forward_grouped(const ltxattn_call* calls, int n_calls, ltxattn_stream_t stream_) {
+  if (!calls || n_calls < 1) return LTXATTN_ERR_INVALID_ARG;
+  if (n_calls > LTXATTN_MAX_GROUP) return LTXATTN_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_calls; ++i) {
+    const ltxattn_call& x = calls[i];
+    const int st = validate(x.q, x.k, x.v, x.out, x.q_len, x.kv_len, x.kv_valid_len, x.batch,
+                            x.heads, x.head_dim, x.scale);
+    if (st != LTXATTN_OK) return st;
+  }
+  // no call's output may overlap another call's inputs or output
+  for (int i = 0; i < n_calls; ++i) {
+    const ltxattn_call& x = calls[i];
+    const size_t nx = (size_t)x.batch * x.q_len * x.heads * x.head_dim * 2;
+    for (int j = 0; j < n_calls; ++j) {
+      if (j == i) continue;
+      const ltxattn_call& y = calls[j];
+      const size_t row = (size_t)y.heads * y.head_dim * 2;
+      const size_t nq = (size_t)y.batch * y.q_len * row, nkv = (size_t)y.batch * y.kv_len * row;
+      if (overlaps(x.out, nx, y.q, nq) || overlaps(x.out, nx, y.k, nkv) ||
+          overlaps(x.out, nx, y.v, nkv) || overlaps(x.out, nx, y.out, nq))
+        return LTXATTN_ERR_INVALID_ARG;
+    }
+  }
+  int st;
+  Context* c = current_context(&st);
+  if (!c) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  ltx::A2vArgs group{};
+  for (int i = 0; i < n_calls; ++i) {
+    const ltxattn_call& x = calls[i];
+    FwdParams p = call_params(*c, x.q_len, x.kv_len, x.kv_valid_len, x.batch, x.heads, x.scale);
+    plan_kernel(p, x.head_dim, 0, c->num_sms, 0);
+    if (!a2v_eligible(p, x.head_dim)) {
+      st = forward_one(c, x.q, x.k, x.v, x.out, x.q_len, x.kv_len, x.kv_valid_len, x.batch,
+                       x.heads, x.head_dim, x.scale, 0, nullptr, stream);
+      if (st != LTXATTN_OK) return st;
+      continue;
+    }
+    CUtensorMap tq, tk, tv, to;
+    if (!encode_bshd(*c, &tq, x.q, x.q_len, x.batch, x.heads, x.head_dim) ||
+        !encode_bshd(*c, &tk, x.k, x.kv_len, x.batch, x.heads, x.head_dim) ||
+        !encode_bshd(*c, &tv, x.v, x.kv_len, x.batch, x.heads, x.head_dim) ||
+        !encode_bshd(*c, &to, x.out, x.q_len, x.batch, x.heads, x.head_dim))
+      return LTXATTN_ERR_CUDA;
+    a2v_append(group, tq, tk, tv, to, p);
+    if (group.n_problems == ltx::kA2vMaxProblems) {
+      if (launch_a2v(group, c->num_sms, stream) != cudaSuccess) return LTXATTN_ERR_CUDA;
+      group = ltx::A2vArgs{};
+    }
+  }
+  if (group.n_problems > 0 && launch_a2v(group, c->num_sms, stream) != cudaSuccess)
+    return LTXATTN_ERR_CUDA;
+  return LTXATTN_OK;
 }
 
 int ltxattn_forward(const void* q, const void* k, const void* v, void* out, int q_len, int kv_len,

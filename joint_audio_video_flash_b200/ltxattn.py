@@ -57,6 +57,7 @@ def load() -> ctypes.CDLL:
             lib.ltxattn_na3d_forward.argtypes = [vp, vp, vp, vp] + [ci] * 9 + [cf, vp]
             lib.ltxattn_forward_partial.argtypes = [vp, vp, vp, vp, vp] + [ci] * 6 + [cf, vp]
             lib.ltxattn_combine.argtypes = [vp, vp, vp] + [ci] * 5 + [vp]
+            lib.ltxattn_forward_grouped.argtypes = [vp, ci, vp]
             lib.ltxattn_entry_point_name.argtypes = [ci]
             lib.ltxattn_entry_point_name.restype = ctypes.c_char_p
             _lib = lib
@@ -153,6 +154,42 @@ def forward(q, k, v, out=None, *, kv_valid_len: int | None = None, scale: float 
         int(num_splits), ctypes.byref(used), ctypes.c_void_p(_stream_handle(stream)))
     _check(st, "ltxattn_forward")
     return (out, used.value) if return_splits else out
+
+
+class _Call(ctypes.Structure):
+    """``ltxattn_call`` of include/ltxattn.h."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("q_len", ctypes.c_int), ("kv_len", ctypes.c_int),
+                ("kv_valid_len", ctypes.c_int), ("batch", ctypes.c_int),
+                ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+def forward_grouped(calls, *, stream=None):
+    """Several independent attention calls through ``ltxattn_forward_grouped``.
+
+    ``calls``: a sequence of dicts with keys q, k, v, out (tensors as for ``forward``; out
+    required) and optional kv_valid_len and scale.  Calls at head_dim 64 whose valid keys
+    fit in one 128-key tile (a2v, audio self-attention) share one launch.  Returns the
+    list of outputs.
+    """
+    arr = (_Call * len(calls))()
+    outs = []
+    for i, c in enumerate(calls):
+        q, k, v, out = c["q"], c["k"], c["v"], c["out"]
+        _check_attention_tensors(q, k, v, out)
+        batch, q_len, heads, head_dim = q.shape
+        kv_len = k.shape[1]
+        kv_valid = c.get("kv_valid_len")
+        scale = c.get("scale")
+        arr[i] = _Call(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), int(q_len),
+                       int(kv_len), int(kv_len if kv_valid is None else kv_valid), int(batch),
+                       int(heads), int(head_dim),
+                       float(1.0 / math.sqrt(head_dim) if scale is None else scale))
+        outs.append(out)
+    st = load().ltxattn_forward_grouped(ctypes.cast(arr, ctypes.c_void_p), len(calls),
+                                        ctypes.c_void_p(_stream_handle(stream)))
+    _check(st, "ltxattn_forward_grouped")
+    return outs
 
 
 def forward_split_noalloc(q, k, v, out, *, kv_valid_len: int | None = None,

@@ -200,3 +200,46 @@ def test_new_calls_reach_cuda_with_valid_arguments(lib):
     assert qk(lib, qo=Q, ko=K) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)  # in place
     assert partial(lib) in (ltxattn.ERR_CUDA, ltxattn.ERR_NOT_INITIALIZED)
     assert comb(lib) == ltxattn.ERR_CUDA
+
+
+def group(lib, *calls):
+    arr = (ltxattn._Call * max(len(calls), 1))()
+    for i, c in enumerate(calls):
+        d = dict(q=Q, k=K, v=V, out=O, q_len=128, kv_len=128, kv_valid_len=126, batch=2,
+                 heads=4, head_dim=64, scale=0.125)
+        d.update(c)
+        arr[i] = ltxattn._Call(**d)
+    return lib.ltxattn_forward_grouped(ctypes.cast(arr, ctypes.c_void_p), len(calls), None)
+
+
+# a second call's tensors, 16 MiB further on
+Q2, K2, V2, O2 = (x + (16 << 20) for x in (Q, K, V, O))
+SECOND = dict(q=Q2, k=K2, v=V2, out=O2)
+
+
+@pytest.mark.parametrize("calls,status", [
+    ((), ltxattn.ERR_INVALID_ARG),                                    # no call
+    (({"q": 0},), ltxattn.ERR_INVALID_ARG),                           # a call's own checks
+    (({}, dict(SECOND, kv_valid_len=0)), ltxattn.ERR_INVALID_ARG),    # ... in any position
+    (({}, dict(SECOND, head_dim=96)), ltxattn.ERR_UNSUPPORTED),
+    (({}, dict(SECOND, k=K2 + 8)), ltxattn.ERR_MISALIGNED),
+    (({}, dict(SECOND, out=O)), ltxattn.ERR_INVALID_ARG),             # two calls write one out
+    (({}, dict(SECOND, out=Q + 4096)), ltxattn.ERR_INVALID_ARG),      # out over another's q
+    (({}, dict(SECOND, q=O)), ltxattn.ERR_INVALID_ARG),               # another reads this out
+    (({}, dict(SECOND, v=O + 1024)), ltxattn.ERR_INVALID_ARG),
+])
+def test_grouped_host_validation(lib, calls, status):
+    assert group(lib, *calls) == status
+
+
+def test_grouped_limits_and_shared_inputs(lib):
+    import torch
+    calls = [dict(q=Q + (i << 24), k=K + (i << 24), v=V + (i << 24), out=O + (i << 24))
+             for i in range(65)]
+    assert group(lib, *calls) == ltxattn.ERR_UNSUPPORTED             # above LTXATTN_MAX_GROUP
+    if torch.cuda.is_available():
+        return
+    # two calls reading the same k and v (a2v and audio self share the audio keys): valid,
+    # so the call gets as far as the context lookup
+    assert group(lib, {}, dict(q=Q2, out=O2)) in (ltxattn.ERR_CUDA,
+                                                   ltxattn.ERR_NOT_INITIALIZED)

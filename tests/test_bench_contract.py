@@ -68,9 +68,14 @@ def test_gpu_arm_line():
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
     e = d["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
-    # four calls per step, one launch each (no key-range parts at these sizes)
-    assert d["gpu_launches"] == 4 * d["steps"]
+    # four calls per step in three launches: audio self-attention and a2v share one grouped
+    # launch (no key-range parts at these sizes)
+    assert d["launch_items"] == [["video_self"], ["audio_self", "a2v"], ["v2a"]]
+    assert d["gpu_launches"] == 3 * d["steps"]
     assert set(d["per_call"]) == {"video_self", "audio_self", "v2a", "a2v"}
+    for name in ("audio_self", "a2v"):
+        g = d["per_call"][name]["group"]
+        assert g["members"] == ["audio_self", "a2v"] and g["us_median"] > 0
     for name, pc in d["per_call"].items():  # the timed outputs against the oracle
         par = pc["parity"]
         assert par["finite"] and par["max_abs"] <= 2e-2 and par["rel_l2"] <= 5e-3, (name, par)
@@ -133,3 +138,17 @@ def test_gpu_arm_context_parallel_line():
     for name, par in d["parity"].items():
         assert par["finite"] and par["max_abs"] <= 2e-2 and par["rel_l2"] <= 5e-3, (name, par)
     assert d["gpu_launches"] == 4 * d["steps"]  # one shard: partial + merge, v2a: partial + merge
+
+
+def test_launch_items_group_the_one_tile_head_dim_64_calls():
+    import bench
+    from joint_audio_video_flash_b200 import workloads
+    _, calls = workloads.configs()["block768"]
+    assert bench.launch_items(calls) == [[0], [1, 3], [2]]
+    assert bench.launch_items(calls, grouped=False) == [[0], [1], [2], [3]]
+    # the long clip's audio side has 252 valid keys (two tiles): nothing to group
+    _, calls = workloads.configs()["longclip"]
+    assert bench.launch_items(calls) == [[0], [1], [2], [3]]
+    assert bench.item_launches([1, 3], [1, 1, 4, 1]) == 1
+    assert bench.item_launches([2], [1, 1, 4, 1]) == 2      # key split + merge
+    assert bench.item_launches(list(range(6)), [1] * 6) == 2  # four calls per launch
