@@ -48,11 +48,11 @@ KERNEL_SOURCES = {
                     "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
 }
 TRAFFIC = {
-    "video_self": {"src": "9e0788ef9aa32a30", "bytes_per_token": (201.6576e6 + 46.488064e6) / 8192,
+    "video_self": {"src": "d7db73ee711fe8cc", "bytes_per_token": (201.593344e6 + 49.534464e6) / 8192,
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
-    "qk_prologue": {"src": "bae7009a0da1dbb0", "bytes": 511.301376e6 + 445.781504e6,
+    "qk_prologue": {"src": "34da3ff698cece0a", "bytes": 511.279104e6 + 446.394624e6,
                     "note": "full launch, B2 x 15360 x 32 x 128, q and k"},
-    "na3d_decoder": {"src": "9c3bbc608b6ea562", "bytes": 802.646272e6 + 248.344064e6,
+    "na3d_decoder": {"src": "6933473e99fe99e5", "bytes": 802.427392e6 + 249.421312e6,
                      "note": "full launch, 16x34x60 grid, 3x7x7 window, 32x128"},
 }
 
