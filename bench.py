@@ -38,7 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, keyed by
 # the hash of the sources that make up that kernel; reported as null once they change.
 KERNEL_SOURCES = {
-    "video_self": ("joint_audio_video_flash_b200/csrc/attn_fwd_pp.cuh",
+    "video_self": ("joint_audio_video_flash_b200/csrc/attn_fwd_pair.cuh",
+                   "joint_audio_video_flash_b200/csrc/attn_fwd_pp.cuh",
                    "joint_audio_video_flash_b200/csrc/attn_fwd.cuh",
                    "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
     "na3d_decoder": ("joint_audio_video_flash_b200/csrc/na3d_fwd.cuh",
@@ -68,6 +69,8 @@ def kernel_label(c, num_sms: int = 148, grouped: bool = False) -> str:
         return f"ltx_attn_fwd_skv<{c.head_dim}, {kt}> (persistent, K/V resident)"
     if c.head_dim == 64 and kt > 2 and qt <= 1:
         return "ltx_attn_fwd<64, 1 S buffer> (two CTAs per SM)"
+    if c.head_dim == 128 and qt >= 8 and (kt < 4 or c.batch * c.heads * ((qt + 1) // 2) >= num_sms):
+        return "ltx_attn_fwd_pair (CTA pairs, cta_group::2, four query tiles per pair)"
     if qt >= 2:
         return f"ltx_attn_fwd_pp<{c.head_dim}> (two 128-row query tiles per CTA)"
     return f"ltx_attn_fwd<{c.head_dim}>"

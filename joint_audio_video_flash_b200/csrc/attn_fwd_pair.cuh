@@ -328,7 +328,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(bar0(L::bPF + part * 2 + g));
+        // default (CTA-scope) release: the cluster-scope form cost each half of P several
+        // hundred cycles and made this kernel slower than the one-SM kernel
+        if (lane == 0) mbar_arrive_remote(bar0(L::bPF + part * 2 + g));
       }
       l_run += (la.x + la.y) + (lb.x + lb.y);
     }

@@ -490,7 +490,7 @@ bool plan_kernel(FwdParams& p, int head_dim, int num_splits, int num_sms, int ma
 }
 
 // Query sides of at least this many 128-row tiles at head_dim 128 (unsplit) run on CTA pairs.
-constexpr int kPairMinQTiles = 1 << 30;  // not dispatched: slower per cycle (see the trace notes)
+constexpr int kPairMinQTiles = 8;
 
 bool use_pair(const FwdParams& p, int head_dim, int num_sms) {
   return head_dim == 128 && p.num_splits == 1 && p.n_q_tiles >= kPairMinQTiles &&

@@ -442,6 +442,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar, uint
                : "memory");
 }
 
+// Arrivals on an mbarrier of either CTA of the pair (`bar` a shared::cluster address) with the
+// instruction's default ordering (release at CTA scope), the form CUTLASS's cluster pipelines
+// use for their cross-CTA arrivals.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
 // try_wait with acquire at cluster scope (the arrivals may come from the other CTA).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
