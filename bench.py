@@ -49,7 +49,7 @@ KERNEL_SOURCES = {
                     "joint_audio_video_flash_b200/csrc/sm100_ptx.cuh"),
 }
 TRAFFIC = {
-    "video_self": {"src": "d7db73ee711fe8cc", "bytes_per_token": (201.593344e6 + 49.534464e6) / 8192,
+    "video_self": {"src": "7c8cf86aca84f424", "bytes_per_token": (201.467392e6 + 47.959040e6) / 8192,
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
     "qk_prologue": {"src": "34da3ff698cece0a", "bytes": 511.279104e6 + 446.394624e6,
                     "note": "full launch, B2 x 15360 x 32 x 128, q and k"},
