@@ -168,7 +168,8 @@ def test_forced_key_splits_two_query_tiles(oracle, d, splits):
     assert_parity(got, ref, f"d={d} splits={splits}")
 
 
-@pytest.mark.parametrize("lq,d,splits", [(130, 128, 0), (100, 64, 1), (100, 64, 2)])
+@pytest.mark.parametrize("lq,d,splits", [(130, 128, 0), (100, 64, 1), (100, 64, 2),
+                                         (1100, 128, 1)])  # the last: the CTA-pair kernel
 def test_growing_scores_force_rescales(oracle, lq, d, splits):
     # keys ordered so that the running max grows tile after tile (exercises the O rescale)
     q, k, v = synth.make_qkv(1, lq, 1024, 2, d, seed=8)
