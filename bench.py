@@ -96,6 +96,24 @@ def launch_items(calls, grouped: bool = True):
     return items
 
 
+def group_base(item, member_us):
+    """The member of a grouped launch whose own launch takes longest: the base of the split."""
+    return max(item, key=lambda i: statistics.median(member_us[("alone", i)]))
+
+
+def group_share(item, i, member_us, groups):
+    """Per-step times of call i's share of its grouped launch, from the interleaved loop: every
+    member but the base gets what it adds (the group minus the group without it, step by
+    step), the base the rest (the group minus the others' additions), so that the shares add
+    up to the group."""
+    group = member_us[("group", groups.index(item))]
+    added = {x: [g - w for g, w in zip(group, member_us[("without", x)])] for x in item}
+    base = group_base(item, member_us)
+    if i != base:
+        return added[i]
+    return [g - sum(added[x][s] for x in item if x != base) for s, g in enumerate(group)]
+
+
 def item_launches(item, splits):
     """Kernel launches of one launch item (a grouped item: one per GROUP_MAX calls)."""
     if len(item) > 1:
@@ -853,25 +871,29 @@ def run_ltxattn(args):
     for i, c in enumerate(calls):
         j = item_of[i]
         grouped = len(items[j]) > 1
-        us_list = member_us[("alone", i)] if grouped else item_us[j]
+        us_list = group_share(items[j], i, member_us, groups) if grouped else item_us[j]
         entry = dist_stats(us_list)
         entry.update(call_roofline(c.flops, c.bytes, entry["us_median"], peaks))
         entry.update({
             "shape": f"B{c.batch} Lq{c.q_len} Lkv{c.kv_len} valid{c.kv_valid_len} "
                      f"H{c.heads} D{c.head_dim}",
-            "splits": splits[i], "kernel": kernel_label(c)})
-        if grouped:  # us_* above: the call alone (its own launch), timed after the step
+            "splits": splits[i],
+            "kernel": kernel_label(c, grouped=True) if grouped else kernel_label(c)})
+        if grouped:
+            # us_* above: this call's share of the grouped launch (group_share); measured in
+            # the interleaved loop after the timed step, L2 flushed before every call
             group_alone = statistics.median(member_us[("group", groups.index(items[j]))])
             without = statistics.median(member_us[("without", i)])
-            entry["timed_alone"] = True
             entry["group"] = {
                 "members": [calls[x].name for x in items[j]],
-                "kernel": kernel_label(c, grouped=True),
+                "share": "base" if group_base(items[j], member_us) == i else "added",
                 "us_median_in_step": statistics.median(item_us[j]),  # the timed step
-                # the next three from the interleaved loop after the step (L2 flushed)
                 "us_median": group_alone,
                 "us_without_this_call": without,
-                "us_added_by_this_call": group_alone - without}
+                "us_added_by_this_call": group_alone - without,
+                # the call on a launch of its own (its own kernel choice)
+                "us_median_own_launch": statistics.median(member_us[("alone", i)]),
+                "kernel_own_launch": kernel_label(c)}
         if c.flops / c.bytes > 1000:  # tensor-bound: time beside the SM clock it ran at
             entry["clock"] = clock_normalised(item_us[j], item_wall[j], trace)
         if rank == 0 and not args.no_parity:  # the oracle on sampled rows, after the timing

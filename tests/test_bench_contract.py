@@ -152,3 +152,18 @@ def test_launch_items_group_the_one_tile_head_dim_64_calls():
     assert bench.item_launches([1, 3], [1, 1, 4, 1]) == 1
     assert bench.item_launches([2], [1, 1, 4, 1]) == 2      # key split + merge
     assert bench.item_launches(list(range(6)), [1] * 6) == 2  # four calls per launch
+
+
+def test_group_share_splits_the_grouped_launch():
+    import bench
+    # interleaved loop: group 80-82 µs; without audio self (index 1) 77-78; without a2v (3) 12-13
+    mu = {("group", 0): [80.0, 82.0, 81.0],
+          ("alone", 1): [10.0, 10.0, 11.0], ("alone", 3): [70.0, 71.0, 70.0],
+          ("without", 1): [77.0, 78.0, 77.0], ("without", 3): [12.0, 12.0, 13.0]}
+    item = [1, 3]
+    assert bench.group_base(item, mu) == 3                     # a2v: the longer own launch
+    audio = bench.group_share(item, 1, mu, [item])
+    a2v = bench.group_share(item, 3, mu, [item])
+    assert audio == [3.0, 4.0, 4.0]                            # what audio self adds
+    assert a2v == [77.0, 78.0, 77.0]                           # the rest of the group
+    assert [x + y for x, y in zip(audio, a2v)] == mu[("group", 0)]
