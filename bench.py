@@ -51,9 +51,9 @@ KERNEL_SOURCES = {
 TRAFFIC = {
     "video_self": {"src": "7c8cf86aca84f424", "bytes_per_token": (201.467392e6 + 47.959040e6) / 8192,
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
-    "qk_prologue": {"src": "34da3ff698cece0a", "bytes": 511.279104e6 + 446.394624e6,
+    "qk_prologue": {"src": "75b060c4d34193c3", "bytes": 511.267584e6 + 446.194176e6,
                     "note": "full launch, B2 x 15360 x 32 x 128, q and k"},
-    "na3d_decoder": {"src": "6933473e99fe99e5", "bytes": 802.427392e6 + 249.421312e6,
+    "na3d_decoder": {"src": "c21ac3fae3c2709b", "bytes": 802.365952e6 + 250.495488e6,
                      "note": "full launch, 16x34x60 grid, 3x7x7 window, 32x128"},
 }
 

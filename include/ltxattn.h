@@ -155,7 +155,9 @@ typedef struct ltxattn_call {
  * self-attention is so small (one query tile per head) that its own launch costs more than
  * its work.  Here such calls (head_dim 64, kv_valid_len <= 128) share one persistent launch,
  * up to four per launch, their (batch, query tile, head) units walked as one sequence by all
- * SMs; every other call runs as ltxattn_forward runs it, in the order given.
+ * SMs, the calls with the most units first; every other call runs as ltxattn_forward runs it,
+ * in the order given, ahead of the shared launches (the calls are independent, so the order
+ * does not change any result).
  *
  *   calls    host array of n_calls descriptors (read during the call only; the pointers in
  *            it are device pointers, as for ltxattn_forward)

@@ -722,17 +722,32 @@ int ltxattn_forward_grouped(const ltxattn_call* calls, int n_calls, ltxattn_stre
   Context* c = current_context(&st);
   if (!c) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  ltx::A2vArgs group{};
+  // the calls the grouped kernel takes, launched after the others, largest first (measured
+  // faster than small problems first: a2v ahead of audio self-attention)
+  struct Grouped {
+    long long units;
+    int call;
+  } grouped[LTXATTN_MAX_GROUP];
+  int n_grouped = 0;
   for (int i = 0; i < n_calls; ++i) {
     const ltxattn_call& x = calls[i];
     FwdParams p = call_params(*c, x.q_len, x.kv_len, x.kv_valid_len, x.batch, x.heads, x.scale);
     plan_kernel(p, x.head_dim, 0, c->num_sms, 0);
-    if (!a2v_eligible(p, x.head_dim)) {
-      st = forward_one(c, x.q, x.k, x.v, x.out, x.q_len, x.kv_len, x.kv_valid_len, x.batch,
-                       x.heads, x.head_dim, x.scale, 0, nullptr, stream);
-      if (st != LTXATTN_OK) return st;
+    if (a2v_eligible(p, x.head_dim)) {
+      grouped[n_grouped++] = {(long long)p.batch * p.heads * p.n_q_tiles, i};
       continue;
     }
+    st = forward_one(c, x.q, x.k, x.v, x.out, x.q_len, x.kv_len, x.kv_valid_len, x.batch,
+                     x.heads, x.head_dim, x.scale, 0, nullptr, stream);
+    if (st != LTXATTN_OK) return st;
+  }
+  std::stable_sort(grouped, grouped + n_grouped,
+                   [](const Grouped& x, const Grouped& y) { return x.units > y.units; });
+  ltx::A2vArgs group{};
+  for (int g = 0; g < n_grouped; ++g) {
+    const ltxattn_call& x = calls[grouped[g].call];
+    FwdParams p = call_params(*c, x.q_len, x.kv_len, x.kv_valid_len, x.batch, x.heads, x.scale);
+    plan_kernel(p, x.head_dim, 0, c->num_sms, 0);
     CUtensorMap tq, tk, tv, to;
     if (!encode_bshd(*c, &tq, x.q, x.q_len, x.batch, x.heads, x.head_dim) ||
         !encode_bshd(*c, &tk, x.k, x.kv_len, x.batch, x.heads, x.head_dim) ||
