@@ -873,7 +873,11 @@ def run_ltxattn(args):
         grouped = len(items[j]) > 1
         us_list = group_share(items[j], i, member_us, groups) if grouped else item_us[j]
         entry = dist_stats(us_list)
-        entry.update(call_roofline(c.flops, c.bytes, entry["us_median"], peaks))
+        added = grouped and group_base(items[j], member_us) != i
+        # a member that rides in another call's launch adds too little time for a throughput
+        # figure to mean anything: its roofline fields are left out
+        if not added:
+            entry.update(call_roofline(c.flops, c.bytes, entry["us_median"], peaks))
         entry.update({
             "shape": f"B{c.batch} Lq{c.q_len} Lkv{c.kv_len} valid{c.kv_valid_len} "
                      f"H{c.heads} D{c.head_dim}",
