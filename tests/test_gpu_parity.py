@@ -381,6 +381,8 @@ PAIR_SHAPES = [
     (1, 2, 1280, 128, 77),       # one key tile, 77 valid keys (too few query tiles for the
                                  # persistent short-key kernel)
     (2, 2, 1536, 4096, 4000),    # many key tiles, masked tail
+    (1, 48, 2100, 300, 290),     # 240 items over at most 74 persistent pairs, three key
+                                 # tiles, ragged query and key tails
 ]
 
 
