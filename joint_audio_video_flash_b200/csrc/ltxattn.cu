@@ -232,8 +232,8 @@ cudaError_t launch_skv(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        cudaStream_t stream) {
   const long long total = (long long)p.batch * p.heads * p.n_q_tiles;
   const int grid = (int)std::min<long long>(total, num_sms);
-  // head_dim 64, one key tile (a2v): three warpgroups doing softmax and epilogue of every
-  // third unit, per-unit K/V and the strided (batch, query tile, head) walk
+  // head_dim 64, one key tile (a2v): per-unit K/V and the strided (batch, query tile, head)
+  // walk, two softmax warpgroups and an epilogue warpgroup
   if (a2v_eligible(p, head_dim)) {
     ltx::A2vArgs a{};
     a2v_append(a, tq, tk, tv, to, p);
