@@ -15,28 +15,38 @@
 // keys starting at the box's corner (one 5-D TMA box each, zero fill past the grid), so a
 // query brick meets nt * ny * nx key tiles.  The key tile's shape is chosen apart from the
 // query brick's, to cover the box with as few tiles as possible (a 2 x 8 x 8 brick's box
-// for a 3 x 7 x 7 window, 4 x 14 x 14, takes seven 4 x 2 x 16 tiles but eight 2 x 8 x 8).  The scores of every tile are masked per
-// element against the query row's own window (a bias of 0 or -inf per key column and per
-// (t, y) row of the tile, from three bit masks, one per axis), and a warp skips the
-// exponentials of each 32-key chunk that lies outside all of its rows' windows.
+// for a 3 x 7 x 7 window, 4 x 14 x 14, takes seven 4 x 2 x 16 tiles but eight 2 x 8 x 8).
+// The scores of every tile are masked per element against the query row's own window:
+// a bias of 0 or -inf per key column x, and per (t, y) row of the tile a choice between the
+// row's max offset and -inf in the exponent (three bit masks, one per axis); a warp skips
+// the exponentials of each 32-key chunk that lies outside all of its rows' windows.
+//
+// Two softmax warpgroups split every key tile: group 0 takes its keys [0, 64), group 1 its
+// keys [64, 128).  Each keeps its own running max, row sum and O accumulator (two PV
+// products per tile, one per half of the keys), so the groups never wait for each other
+// inside a brick and every SM sub-partition runs two softmax warps; the halves are merged
+// once per brick (the group-0 statistics go to group 1 through shared memory, group 1
+// writes both halves' weights, the epilogue sums the two O's with them).
 // Softmax and epilogue warps arrive on their mbarriers once per warp, after __syncwarp.
 //
 // Persistent: one CTA per SM takes every gridDim.x-th (batch, head, brick) unit:
 //   warp 0      TMA producer: Q bricks (2 stages, the next brick's Q issued with the
-//               current brick's first K), K and V tiles through rings (K before V);
+//               current brick's last K), K and V tiles through rings (K before V);
 //   warp 1      MMA issuer (elected lane): S = Q K^T into one of two S buffers, then
-//               O += P V of the previous tile (possibly the previous brick) into one of
-//               two O buffers (brick i uses O buffer i % 2);
-//   warps 4-7   softmax, one query row per thread: window mask, online softmax with the
-//               lazy O rescale (only when a row's max grows by > 2^8; a row that has
-//               seen no key yet takes its first max without touching O, which is still
-//               zero), P written over S as bf16; at a brick's end its row sums l go to
-//               shared memory;
-//   warps 8-11  epilogue: waits for a brick's O and l, frees the O buffer, divides by l,
-//               rounds to bf16, stages the brick and stores it with one 5-D TMA store
-//               (clipped at the grid's edges), overlapping the next brick's MMAs.
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D).
-// Registers (setmaxnreg): producer/MMA warpgroup 80, softmax 232, epilogue 128.
+//               O_g += P_g V_g of the previous tile (possibly the previous brick) for each
+//               half g once its group has written P;
+//   warps 4-11  softmax, two groups of four warps, one query row per thread and group:
+//               window mask, online softmax with the lazy O rescale (only when a row's max
+//               grows by > 2^8; a row that has seen no key yet takes its first max without
+//               touching O, which is still zero), P written over its half of S as bf16;
+//   warps 12-15 epilogue: waits for a brick's O's and weights, frees the O buffers, merges
+//               the halves, rounds to bf16, stages the brick in its own Q stage and stores
+//               it with one 5-D TMA store (clipped at the grid's edges), overlapping the
+//               next brick's MMAs; the Q stage returns to the producer once the store has
+//               read it.
+// TMEM (512 columns): S0 [0,128), S1 [128,256); from 256 the O accumulators, one per group
+// (head_dim 128), or one per group and brick parity (head_dim 64: 4 x 64 columns).
+// Registers (setmaxnreg): producer/MMA warpgroup 88, softmax 168 (each group), epilogue 88.
 #pragma once
 
 #include "attn_fwd.cuh"
@@ -55,13 +65,14 @@ struct Na3dParams {
   unsigned long long timeout_ns;
 };
 
-constexpr int kNaThreads = 384;
-constexpr int kNaRegsLaunch = 168;  // what ptxas gives a 384-thread, 1-CTA kernel
-constexpr int kNaRegsIssue = 80;    // warps 0-3
-constexpr int kNaRegsSoftmax = 232; // warps 4-7
-constexpr int kNaRegsEpi = 128;     // warps 8-11
-static_assert(128 * (kNaRegsIssue + kNaRegsSoftmax + kNaRegsEpi) <= kNaThreads * kNaRegsLaunch,
+constexpr int kNaThreads = 512;
+constexpr int kNaRegsLaunch = 128;  // what ptxas gives a 512-thread, 1-CTA kernel
+constexpr int kNaRegsIssue = 88;    // warps 0-3
+constexpr int kNaRegsSoftmax = 168; // warps 4-11
+constexpr int kNaRegsEpi = 88;      // warps 12-15
+static_assert(128 * (kNaRegsIssue + 2 * kNaRegsSoftmax + kNaRegsEpi) <= kNaThreads * kNaRegsLaunch,
               "register split exceeds the launch allocation");
+constexpr int kNaHalf = kBlockN / 2;  // keys of a tile per softmax group
 
 template <int D>
 struct NaSmem {
@@ -69,35 +80,43 @@ struct NaSmem {
   static constexpr int kBoxes = D / 64;            // 64-column (128-byte) boxes per row
   static constexpr int kBoxBytes = kBlockM * 128;  // 128 rows x 64 bf16
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  // the epilogue stages a brick's output in the brick's own Q stage (its MMAs are done)
   static constexpr int kQStages = 2;
   static constexpr int kKStages = D == 64 ? 4 : 2;
-  static constexpr int kVStages = D == 64 ? 4 : 2;
-  static constexpr int kStaging = D == 64 ? 2 : 1;  // output staging bricks
+  static constexpr int kVStages = D == 64 ? 4 : 3;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQStages * kTileBytes;
   static constexpr int kV = kK + kKStages * kTileBytes;
-  static constexpr int kStage = kV + kVStages * kTileBytes;
-  static constexpr int kRowSum = kStage + kStaging * kTileBytes;  // l per O buffer and row
-  static constexpr int kBar = kRowSum + 2 * kBlockM * 4;
+  // one slot of per-row brick statistics: group 0's (max, sum), which group 1 replaces by
+  // the two halves' merge weights
+  static constexpr int kStats = kV + kVStages * kTileBytes;
+  static constexpr int kBar = kStats + kBlockM * 8;
   static constexpr int bQF = 0;
-  static constexpr int bQE = bQF + kQStages;
+  static constexpr int bQE = bQF + kQStages;  // Q stage free: the brick's output store read it
   static constexpr int bKF = bQE + kQStages;
   static constexpr int bKE = bKF + kKStages;
   static constexpr int bVF = bKE + kKStages;
   static constexpr int bVE = bVF + kVStages;
   static constexpr int bSF = bVE + kVStages;  // 2: scores in S buffer
-  static constexpr int bPF = bSF + 2;         // 2: P in S buffer (128 arrivals)
-  static constexpr int bOF = bPF + 2;         // 2: a brick's last PV done in O buffer
-  static constexpr int bOE = bOF + 2;         // 2: O buffer and its row sums read (128)
-  static constexpr int bLF = bOE + 2;         // 2: row sums of a brick written (128)
-  static constexpr int bOD = bLF + 2;         // every PV
-  static constexpr int bDrain = bOD + 1;
+  static constexpr int bPF = bSF + 2;         // 2 x 2: P of group g in S buffer (4 warps)
+  static constexpr int bOF = bPF + 4;         // 2: a brick's last PVs done (by brick parity)
+  static constexpr int bOE = bOF + 2;         // 2: a brick's O's and weights read (4 warps)
+  static constexpr int bSA = bOE + 2;         // group 0's statistics of a brick written
+  static constexpr int bLF = bSA + 1;         // merge weights of a brick written
+  static constexpr int bOD = bLF + 1;         // 2: every PV of group g
+  static constexpr int bDrain = bOD + 2;
   static constexpr int kNumBars = bDrain + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kUsed = kAbort + 4;
   static constexpr int kAlloc = ((kUsed + 1024 + 1023) / 1024) * 1024;
+  // O accumulators: one per group, and per brick parity where they fit (head_dim 64)
+  static constexpr int kOBufs = D == 64 ? 2 : 1;
   static constexpr uint32_t kColO = 256;
+  static_assert(kColO + 2 * kOBufs * D <= 512, "TMEM columns");
+  __device__ __forceinline__ static uint32_t col_o(int g, int brick) {
+    return kColO + (uint32_t)(((brick % kOBufs) * 2 + g) * D);
+  }
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -177,7 +196,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + L::kBar + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
-  float* row_sum = reinterpret_cast<float*>(smem + L::kRowSum);
+  float2* stats = reinterpret_cast<float2*>(smem + L::kStats);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -203,12 +222,14 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::bSF + s), 1);
-      mbar_init(bar(L::bPF + s), 4);
+      mbar_init(bar(L::bPF + 2 * s), 4);
+      mbar_init(bar(L::bPF + 2 * s + 1), 4);
       mbar_init(bar(L::bOF + s), 1);
       mbar_init(bar(L::bOE + s), 4);
-      mbar_init(bar(L::bLF + s), 4);
+      mbar_init(bar(L::bOD + s), 1);
     }
-    mbar_init(bar(L::bOD), 1);
+    mbar_init(bar(L::bSA), 4);
+    mbar_init(bar(L::bLF), 4);
     mbar_init(bar(L::bDrain), 1);
     *abort_flag = (*reinterpret_cast<volatile int*>(p.status) != kDevOk) ? 1 : 0;
     fence_mbar_init();
@@ -264,8 +285,9 @@ __global__ void __launch_bounds__(kNaThreads, 1)
             tma_load_5d(sbase + L::kK + ks * L::kTileBytes + bx * L::kBoxBytes, &tm_k,
                         bar(L::bKF + ks), cur.h * D + bx * 64, kx, ky, kt, cur.b);
           last_k[ks] = g;
-          // the next brick's queries, once this brick's first keys are on their way
-          if (j == 0 && i + 1 < cnt) {
+          // the next brick's queries with this brick's last keys: their stage held the
+          // output of brick i - 1, whose store must have read it
+          if (j == cur.n - 1 && i + 1 < cnt) {
             ok = load_q(i + 1, nxt);
             if (!ok) break;
           }
@@ -311,26 +333,31 @@ __global__ void __launch_bounds__(kNaThreads, 1)
       const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
       const SmemDesc dv = SmemDesc::sw128(sbase + L::kV, L::kBoxBytes, 1024);
       bool issued = false;
-      // O += P_t V_t for key tile t (global count) = tile j of brick i, which has n tiles
+      // O_g += P_g V_g over both halves g of key tile t (global count) = tile j of brick i,
+      // which has n tiles; each half as soon as its group has written P
       auto pv = [&](int t, int i, int j, int n) -> bool {
         const int sb = t & 1;
         const int vs = t % L::kVStages;
-        const int ob = i & 1;
-        if (!wt(bar(L::bPF + sb), (uint32_t)(t >> 1) & 1u) ||
-            !wt(bar(L::bVF + vs), (uint32_t)(t / L::kVStages) & 1u))
+        if (!wt(bar(L::bVF + vs), (uint32_t)(t / L::kVStages) & 1u)) return false;
+        // a brick's first PVs overwrite their O buffers: the epilogue of brick i - kOBufs
+        // read them
+        const int ip = i - L::kOBufs;
+        if (j == 0 && ip >= 0 && !wt(bar(L::bOE + (ip & 1)), (uint32_t)(ip >> 1) & 1u))
           return false;
-        // a brick's first PV overwrites its O buffer: the epilogue of brick i - 2 read it
-        if (j == 0 && i >= 2 && !wt(bar(L::bOE + ob), (uint32_t)((i >> 1) - 1) & 1u))
-          return false;
-        tc_fence_after();
         const uint32_t v_off = (uint32_t)vs * L::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
-          umma_ts_elect(tmem + L::kColO + ob * D, tmem + sb * 128 + kk * 8,
-                        dv.at(v_off + kk * 16 * 128), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!wt(bar(L::bPF + 2 * sb + h), (uint32_t)(t >> 1) & 1u)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kNaHalf / 16; ++kk)
+            umma_ts_elect(tmem + L::col_o(h, i), tmem + sb * 128 + h * kNaHalf + kk * 8,
+                          dv.at(v_off + (h * kNaHalf + kk * 16) * 128), idesc_pv,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_elect(bar(L::bOD + h));
+        }
         umma_commit_elect(bar(L::bVE + vs));
-        umma_commit_elect(bar(L::bOD));
-        if (j == n - 1) umma_commit_elect(bar(L::bOF + ob));
+        if (j == n - 1) umma_commit_elect(bar(L::bOF + (i & 1)));
         return true;
       };
       bool ok = true;
@@ -358,7 +385,6 @@ __global__ void __launch_bounds__(kNaThreads, 1)
           issued = true;
           umma_commit_elect(bar(L::bSF + sb));
           umma_commit_elect(bar(L::bKE + ks));
-          if (j == cur.n - 1) umma_commit_elect(bar(L::bQE + qs));
           if (pt >= 0) ok = pv(pt, pi, pj, pn);
           pt = g;
           pi = i;
@@ -374,9 +400,10 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     }
   } else if (warp < 4) {
     setmaxnreg_dec<kNaRegsIssue>();  // warps 2-3: idle
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ softmax
     setmaxnreg_inc<kNaRegsSoftmax>();
+    const int grp = (warp >> 2) - 1;  // 0: keys [0, 64) of every tile, 1: keys [64, 128)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t tlane = tmem + ((uint32_t)(wq * 32) << 16);
@@ -384,12 +411,15 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     const int lt = row / (BX * BY), ly = (row / BX) % BY, lx = row % BX;
     const float sl2 = p.scale_log2;
     const float2 sc2 = make_float2(sl2, sl2);
+    constexpr int kRows = kNaHalf / KX;   // (t, y) rows of a tile in this group's half
+    constexpr int kRowsChunk = 32 / KX;  // rows per 32-key chunk
+    const int r0 = grp * kRows;          // the half's first row in the tile
     bool ok = !*abort_flag;
     int g = 0;
     Brick cur;
     for (int i = 0; i < cnt && ok; ++i) {
       cur.init(unit(i), p);
-      const int ob = i & 1;
+      const uint32_t tO = tlane + L::col_o(grp, i);
       // window starts of this query (rows past the grid's edge take the last position's
       // window; their output is clipped by the store)
       const int wt0 = na_window_start(min(cur.t0 + lt, p.grid_t - 1), p.win_t, p.grid_t);
@@ -402,45 +432,57 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(g >> 1) & 1u, ctl));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tS = tlane + sb * 128;
-        float s[kBlockN];
-#pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c)
-          tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+        const uint32_t tS = tlane + sb * 128 + grp * kNaHalf;
+        float s[kNaHalf];
+        tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
         int kt, ky, kx;
         cur.key_origin(j, kt, ky, kx);
         const uint32_t mt = na_bits(wt0 - kt, wt0 - kt + p.win_t, KT);
         const uint32_t my = na_bits(wy0 - ky, wy0 - ky + p.win_y, KY);
         const uint32_t mx = na_bits(wx0 - kx, wx0 - kx + p.win_x, KX);
-        // window mask as additive biases (0 inside, -inf outside): one per key column x
-        // of the tile and one per (t, y) row of it, two packed adds per pair of scores
+        // the key columns x of the tile outside this query's window: a bias of -inf, one
+        // packed add per pair of scores
         float2 bx2[KX / 2];
 #pragma unroll
         for (int c2 = 0; c2 < KX / 2; ++c2)
           bx2[c2] = make_float2((mx >> (2 * c2)) & 1u ? 0.0f : -INFINITY,
                                 (mx >> (2 * c2 + 1)) & 1u ? 0.0f : -INFINITY);
-        uint32_t rows_in = 0;  // (t, y) rows of the tile inside this query's window
-        tmem_ld_wait();
+        uint32_t rows_in = 0;  // (t, y) rows of the half inside this query's window
 #pragma unroll
-        for (int r = 0; r < KT * KY; ++r) {
-          const bool in = (mt >> (r / KY)) & (my >> (r % KY)) & 1u;
-          rows_in |= (in ? 1u : 0u) << r;
-          const float rb = in ? 0.0f : -INFINITY;
-          const float2 rb2 = make_float2(rb, rb);
+        for (int r = 0; r < kRows; ++r) {
+          const int rr = r0 + r;
+          rows_in |= ((mt >> (rr / KY)) & (my >> (rr % KY)) & 1u) << r;
+        }
+        if (mx == 0) rows_in = 0;
+        tmem_ld_wait();
+        // the max over the keys inside the window: per row of the half over its
+        // column-masked scores, rows outside the window left out
+        float mrow = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          float* sr = &s[r * KX];
 #pragma unroll
           for (int c2 = 0; c2 < KX / 2; ++c2) {
-            float2 v = make_float2(s[r * KX + 2 * c2], s[r * KX + 2 * c2 + 1]);
-            v = __fadd2_rn(__fadd2_rn(v, bx2[c2]), rb2);
-            s[r * KX + 2 * c2] = v.x;
-            s[r * KX + 2 * c2 + 1] = v.y;
+            const float2 v = __fadd2_rn(make_float2(sr[2 * c2], sr[2 * c2 + 1]), bx2[c2]);
+            sr[2 * c2] = v.x;
+            sr[2 * c2 + 1] = v.y;
           }
+          float a = fmaxf(sr[0], sr[1]), b = fmaxf(sr[2], sr[3]);
+#pragma unroll
+          for (int c = 4; c + 4 <= KX; c += 4) {
+            a = fmax3(a, sr[c], sr[c + 1]);
+            b = fmax3(b, sr[c + 2], sr[c + 3]);
+          }
+          mrow = (rows_in >> r) & 1u ? fmax3(mrow, a, b) : mrow;
         }
-        const float mx_t = row_max<kBlockN>(s) * sl2;
+        const float mx_t = mrow * sl2;
         const bool grow = m_run != -INFINITY && mx_t > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, grow)) {
-          // O must hold the PV of the previous tile before it is rescaled (tcgen05.ld/st
-          // are warp-collective: lanes whose max did not grow scale by 1)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOD), (uint32_t)(g - 1) & 1u, ctl));
+          // O must hold this group's PV of the previous tile before it is rescaled
+          // (tcgen05.ld/st are warp-collective: lanes whose max did not grow scale by 1)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(bar(L::bOD + grp), (uint32_t)(g - 1) & 1u, ctl));
           if (!ok) break;
           tc_fence_after();
           const float mn = grow ? mx_t : m_run;
@@ -448,12 +490,12 @@ __global__ void __launch_bounds__(kNaThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            tmem_ld32(tlane + L::kColO + ob * D + c * 32, o);
+            tmem_ld32(tO + c * 32, o);
             tmem_ld_wait();
             uint32_t u[32];
 #pragma unroll
             for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(o[x] * f);
-            tmem_st32(tlane + L::kColO + ob * D + c * 32, u);
+            tmem_st32(tO + c * 32, u);
           }
           tmem_st_wait();
           l_run *= f;
@@ -462,18 +504,32 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         // a row's first keys: take their max (O and l of the row are still zero)
         if (m_run == -INFINITY) m_run = mx_t;
         const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-        const float2 nm2 = make_float2(-m_use, -m_use);
-        float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
-        if (mx == 0) rows_in = 0;
+        // rows outside the window get an exponent offset of -inf (p = 0)
+        float2 nm2[kRows];
 #pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c) {
+        for (int r = 0; r < kRows; ++r) {
+          const float nm = (rows_in >> r) & 1u ? -m_use : -INFINITY;
+          nm2[r] = make_float2(nm, nm);
+        }
+        float2 la = make_float2(0.0f, 0.0f), lb = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int c = 0; c < kNaHalf / 32; ++c) {
           // a 32-key chunk outside every window of this warp's rows: P = 0 without the
-          // exponentials (the MUFU bounds this loop)
-          constexpr int kRowsChunk = 32 / KX;
+          // exponentials
           const uint32_t chunk_rows = (rows_in >> (c * kRowsChunk)) & ((1u << kRowsChunk) - 1u);
           uint32_t pk[16];
           if (__any_sync(0xffffffffu, chunk_rows != 0)) {
-            exp2_pack16(&s[c * 32], sc2, nm2, la, lb, pk);
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const int k = c * 32 + 2 * x;
+              const float2 a = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2[k / KX]);
+              const float2 e = make_float2(ex2(a.x), ex2(a.y));
+              if (x & 1)
+                lb = __fadd2_rn(lb, e);
+              else
+                la = __fadd2_rn(la, e);
+              pk[x] = pack_bf16x2(e.x, e.y);
+            }
           } else {
 #pragma unroll
             for (int x = 0; x < 16; ++x) pk[x] = 0u;
@@ -483,18 +539,34 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::bPF + sb));
+        if (lane == 0) mbar_arrive(bar(L::bPF + 2 * sb + grp));
         l_run += (la.x + la.y) + (lb.x + lb.y);
       }
       if (!ok) break;
-      // the row sums of brick i - 2 in this slot were read by its epilogue
-      if (i >= 2)
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(L::bOE + ob), (uint32_t)((i >> 1) - 1) & 1u, ctl));
-      if (!ok) break;
-      row_sum[ob * kBlockM + row] = l_run;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::bLF + ob));
+      if (grp == 0) {
+        // the slot's previous contents (brick i - 1's weights) were read by its epilogue
+        if (i >= 1)
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bOE + ((i - 1) & 1)),
+                                                 (uint32_t)((i - 1) >> 1) & 1u, ctl));
+        if (!ok) break;
+        stats[row] = make_float2(m_run, l_run);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::bSA));
+      } else {
+        // merge weights of the two halves: O = w0 O_0 + w1 O_1 with w_g = 2^(m_g - m) / l,
+        // m the larger max and l = l_0 2^(m_0 - m) + l_1 2^(m_1 - m)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSA), (uint32_t)i & 1u, ctl));
+        if (!ok) break;
+        const float2 a = stats[row];
+        const float m = fmaxf(a.x, m_run);
+        const float f0 = a.x == -INFINITY ? 0.0f : ex2(a.x - m);
+        const float f1 = m_run == -INFINITY ? 0.0f : ex2(m_run - m);
+        const float l = a.y * f0 + l_run * f1;
+        const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+        stats[row] = make_float2(f0 * inv_l, f1 * inv_l);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::bLF));
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -507,43 +579,42 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     Brick cur;
     for (int i = 0; i < cnt && ok; ++i) {
       cur.init(unit(i), p);
-      const int ob = i & 1;
-      const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-      bool w = mbar_wait(bar(L::bOF + ob), ph, ctl);
-      w = w && mbar_wait(bar(L::bLF + ob), ph, ctl);
+      bool w = mbar_wait(bar(L::bOF + (i & 1)), (uint32_t)(i >> 1) & 1u, ctl);
+      w = w && mbar_wait(bar(L::bLF), (uint32_t)i & 1u, ctl);
       ok = named_bar_and(1, kBlockM, w);  // the four warps leave together or not at all
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.0f / row_sum[ob * kBlockM + row];
-      const int sbuf = L::kStaging == 2 ? (i & 1) : 0;
-      uint8_t* stage = smem + L::kStage + sbuf * L::kTileBytes;
-      // the store issued kStaging bricks ago from this staging buffer must have read it
-      if (leader) tma_store_wait_read<L::kStaging - 1>();
-      named_bar_sync(1, kBlockM);
-      const float2 il2 = make_float2(inv_l, inv_l);
+      const float2 wgt = stats[row];
+      const float2 w0 = make_float2(wgt.x, wgt.x), w1 = make_float2(wgt.y, wgt.y);
+      const uint32_t tO0 = tlane + L::col_o(0, i), tO1 = tlane + L::col_o(1, i);
+      // the output is staged in the brick's Q stage: all of its MMAs are complete
+      const int qs = i % L::kQStages;
+      uint8_t* stage = smem + L::kQ + qs * L::kTileBytes;
 #pragma unroll
-      for (int bx = 0; bx < L::kBoxes; ++bx) {
-        float o[64];
-        tmem_ld32(tlane + L::kColO + ob * D + bx * 64, *reinterpret_cast<float(*)[32]>(&o[0]));
-        tmem_ld32(tlane + L::kColO + ob * D + bx * 64 + 32,
-                  *reinterpret_cast<float(*)[32]>(&o[32]));
+      for (int c = 0; c < D / 32; ++c) {
+        float o0[32], o1[32];
+        tmem_ld32(tO0 + c * 32, o0);
+        tmem_ld32(tO1 + c * 32, o1);
         tmem_ld_wait();
-        if (bx == L::kBoxes - 1) {
+        if (c == D / 32 - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::bOE + ob));
+          if (lane == 0) mbar_arrive(bar(L::bOE + (i & 1)));
         }
+        // 32 columns: half of a 64-column box, four 16-byte units of the swizzled row
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 4; ++u) {
           uint32_t w4[4];
 #pragma unroll
           for (int x = 0; x < 4; ++x) {
-            const float2 v2 =
-                __fmul2_rn(make_float2(o[8 * u + 2 * x], o[8 * u + 2 * x + 1]), il2);
+            const int k = 8 * u + 2 * x;
+            const float2 v2 = __ffma2_rn(make_float2(o0[k], o0[k + 1]), w0,
+                                         __fmul2_rn(make_float2(o1[k], o1[k + 1]), w1));
             w4[x] = pack_bf16x2(v2.x, v2.y);
           }
-          *reinterpret_cast<uint4*>(stage + bx * L::kBoxBytes + row * 128 +
-                                    ((u ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          const int uu = (c & 1) * 4 + u;
+          *reinterpret_cast<uint4*>(stage + (c >> 1) * L::kBoxBytes + row * 128 +
+                                    ((uu ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
       fence_proxy_async_smem();
@@ -551,9 +622,12 @@ __global__ void __launch_bounds__(kNaThreads, 1)
       if (leader) {
 #pragma unroll
         for (int bx = 0; bx < L::kBoxes; ++bx)
-          tma_store_5d(&tm_o, sbase + L::kStage + sbuf * L::kTileBytes + bx * L::kBoxBytes,
+          tma_store_5d(&tm_o, sbase + L::kQ + qs * L::kTileBytes + bx * L::kBoxBytes,
                        cur.h * D + bx * 64, cur.x0, cur.y0, cur.t0, cur.b);
         tma_store_commit();
+        // the stage goes back to the producer once the store has read it
+        tma_store_wait_read<0>();
+        mbar_arrive(bar(L::bQE + qs));
       }
     }
     if (leader) tma_store_wait_read<0>();
