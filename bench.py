@@ -522,7 +522,7 @@ def measure_na3d_config(steps, warmup, peaks, dev, stream):
     ltxattn.check()
     r = dist_stats(us[0])
     flops = na3d_step_flops()
-    issued = na_key_tiles(grid, window) * b * heads * 4.0 * 128 * 128 * d
+    issued = na_issued_flops(grid, window, b, heads, d)
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     tfl = flops / (r["us_median"] * 1e-6) / 1e12
     r.update({"tflops": tfl, "frac_bf16_peak": tfl / burst, "bound": "tensor",
@@ -1177,12 +1177,14 @@ def run_prologue(args):
 
 # (query brick, key tile) pairs the library is built for, as t x y x x
 NA_SHAPES = (((2, 8, 8), (2, 8, 8)), ((2, 8, 8), (4, 2, 16)), ((1, 8, 16), (1, 8, 16)),
-             ((1, 8, 16), (1, 16, 8)), ((4, 4, 8), (4, 4, 8)), ((4, 4, 8), (4, 2, 16)))
+             ((1, 8, 16), (1, 16, 8)), ((4, 4, 8), (4, 4, 8)), ((4, 4, 8), (4, 2, 16)),
+             ((2, 8, 8), (4, 2, 14)))
 
 
 def na_key_tiles(grid, window, with_shape=False):
-    """128-key tiles the neighbourhood kernel multiplies per (batch, head): the shape pair
-    with the fewest, as the library picks it (counting only; no attention math)."""
+    """Key tiles the neighbourhood kernel multiplies per (batch, head), for the shape pair the
+    library picks: the fewest tiles, then the fewest keys in all tiles (counting only; no
+    attention math).  With with_shape, also the query brick and key tile shapes."""
     def start(i, k, n):
         return min(max(i - k // 2, 0), n - k)
 
@@ -1194,9 +1196,21 @@ def na_key_tiles(grid, window, with_shape=False):
             tot += -(-(r1 - r0) // kblk)
         return tot
 
-    best = min((axis(grid[0], qb[0], kb[0], window[0]) * axis(grid[1], qb[1], kb[1], window[1])
-                * axis(grid[2], qb[2], kb[2], window[2]), qb, kb) for qb, kb in NA_SHAPES)
-    return best if with_shape else best[0]
+    best = None
+    for qb, kb in NA_SHAPES:
+        tiles = (axis(grid[0], qb[0], kb[0], window[0]) * axis(grid[1], qb[1], kb[1], window[1])
+                 * axis(grid[2], qb[2], kb[2], window[2]))
+        key = (tiles, tiles * kb[0] * kb[1] * kb[2])
+        if best is None or key < best[0]:
+            best = (key, tiles, qb, kb)
+    return best[1:] if with_shape else best[1]
+
+
+def na_issued_flops(grid, window, b, heads, d):
+    """FLOPs of the tiles the tensor cores multiply: QK^T and PV of every 128-query x
+    (keys per tile) tile."""
+    tiles, _, kb = na_key_tiles(grid, window, with_shape=True)
+    return tiles * b * heads * 4.0 * 128 * (kb[0] * kb[1] * kb[2]) * d
 
 
 def na_kernel_label(grid, window, d):
@@ -1251,8 +1265,7 @@ def run_na3d(args):
     total_ms = max_over_ranks(t0.elapsed_time(t1), world)
     step_flops = na3d_step_flops()
     value = whole_job_tflops(step_flops, args.steps, world, total_ms)
-    tiles = na_key_tiles(grid, window) * b * heads
-    issued = tiles * 4.0 * 128 * 128 * d  # the 128 x 128 tiles the tensor cores multiply
+    issued = na_issued_flops(grid, window, b, heads, d)  # the tiles the tensor cores multiply
     issued_tflops = whole_job_tflops(issued, args.steps, world, total_ms)
     peaks, peak_src = load_peaks()
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))

@@ -372,8 +372,11 @@ int launch_prologue(const ltx::PrologueParams& p, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- neighbourhood attention
-// Query brick and key tile shapes (t x y x x = 128 tokens each) the kernel is built for; the
-// host takes the pair whose bricks meet the fewest key tiles in total.
+// Query brick (t x y x x = 128 tokens) and key tile (112 or 128 keys) shapes the kernel is
+// built for; the host takes the pair whose bricks meet the fewest key tiles in total (a
+// tile's MMAs do not depend on its width), of those the one with the fewest keys (K/V bytes
+// and softmax work).  4 x 2 x 14 tiles cover the 4 x 14 x 14 key box of a 2 x 8 x 8 brick
+// under a 3 x 7 x 7 window exactly: seven tiles of 112 keys instead of seven of 128.
 struct NaShape {
   int bt, by, bx;  // query brick
   int kt, ky, kx;  // key tile
@@ -381,6 +384,7 @@ struct NaShape {
 constexpr NaShape kNaShapes[] = {
     {2, 8, 8, 2, 8, 8}, {2, 8, 8, 4, 2, 16}, {1, 8, 16, 1, 8, 16},
     {1, 8, 16, 1, 16, 8}, {4, 4, 8, 4, 4, 8}, {4, 4, 8, 4, 2, 16},
+    {2, 8, 8, 4, 2, 14},
 };
 constexpr int kNumNaShapes = (int)(sizeof(kNaShapes) / sizeof(kNaShapes[0]));
 
@@ -922,11 +926,13 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
   if (!c) return st;
 
   int best = 0;
-  long long best_tiles = -1;
+  long long best_keys = -1, best_tiles = -1;
   for (int i = 0; i < kNumNaShapes; ++i) {
-    const long long t = na_tiles_total(kNaShapes[i], grid_t, grid_y, grid_x, window_t, window_y,
-                                       window_x);
-    if (best_tiles < 0 || t < best_tiles) {
+    const NaShape& s = kNaShapes[i];
+    const long long t = na_tiles_total(s, grid_t, grid_y, grid_x, window_t, window_y, window_x);
+    const long long keys = t * (s.kt * s.ky * s.kx);
+    if (best_tiles < 0 || t < best_tiles || (t == best_tiles && keys < best_keys)) {
+      best_keys = keys;
       best_tiles = t;
       best = i;
     }

@@ -172,6 +172,15 @@ struct NaBrick {
   }
 };
 
+// Eight 32-bit columns of this warp's TMEM lanes into registers.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
 // Bits [max(lo, 0), min(hi, n)) of a 32-bit word (n <= 32).
 __device__ __forceinline__ uint32_t na_bits(int lo, int hi, int n) {
   const int a = lo > 0 ? lo : 0;
@@ -185,9 +194,15 @@ __global__ void __launch_bounds__(kNaThreads, 1)
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const Na3dParams p) {
   static_assert(BT * BY * BX == kBlockM && BX <= 32 && BY <= 32 && BT <= 32, "brick");
-  static_assert(KT * KY * KX == kBlockN && KT * KY <= 32 && 32 % KX == 0 && KX % 2 == 0,
-                "key tile: 128 keys, rows of KX keys filling whole 32-key chunks");
+  // a key tile of kKeys keys: each softmax group takes kGrpKeys of them (whole rows of KX
+  // keys) and writes their P over a 64-key span, zero past its keys
+  constexpr int kKeys = KT * KY * KX;
+  constexpr int kGrpKeys = kKeys / 2;
+  static_assert(kKeys <= kBlockN && kGrpKeys % KX == 0 && kGrpKeys % 8 == 0 &&
+                    kGrpKeys > kNaHalf - 16 && KT * KY <= 32 && KX % 2 == 0 && KX >= 4,
+                "key tile: 112 to 128 keys, each half whole rows of an even number of keys");
   using L = NaSmem<D>;
+  constexpr uint32_t kKVBytes = (uint32_t)kKeys * 128u * L::kBoxes;  // one K or V tile
   using Brick = NaBrick<BT, BY, BX, KT, KY, KX>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -238,6 +253,15 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     tmem_alloc(sbase + L::kTmemSlot, 512);
     tmem_relinquish();
   }
+  if constexpr (kKeys < kBlockN) {
+    // rows [kKeys, 128) of the V stages are never loaded, and the second group's PV reads
+    // rows up to kGrpKeys + 63 (with P = 0 past its keys): they must hold finite values
+    constexpr int kPad16 = (kBlockN - kKeys) * 128 / 16;  // 16-byte units per box
+    for (int i = threadIdx.x; i < L::kVStages * L::kBoxes * kPad16; i += blockDim.x)
+      *reinterpret_cast<uint4*>(smem + L::kV + (i / kPad16) * L::kBoxBytes + kKeys * 128 +
+                                (i % kPad16) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -279,7 +303,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
           const int ks = g % L::kKStages;
           ok = mbar_wait_lean(bar(L::bKE + ks), ((uint32_t)(g / L::kKStages) & 1u) ^ 1u, ctl);
           if (!ok) break;
-          mbar_arrive_expect_tx(bar(L::bKF + ks), L::kTileBytes);
+          mbar_arrive_expect_tx(bar(L::bKF + ks), kKVBytes);
 #pragma unroll
           for (int bx = 0; bx < L::kBoxes; ++bx)
             tma_load_5d(sbase + L::kK + ks * L::kTileBytes + bx * L::kBoxBytes, &tm_k,
@@ -294,7 +318,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
           const int vs = g % L::kVStages;
           ok = mbar_wait_lean(bar(L::bVE + vs), ((uint32_t)(g / L::kVStages) & 1u) ^ 1u, ctl);
           if (!ok) break;
-          mbar_arrive_expect_tx(bar(L::bVF + vs), L::kTileBytes);
+          mbar_arrive_expect_tx(bar(L::bVF + vs), kKVBytes);
 #pragma unroll
           for (int bx = 0; bx < L::kBoxes; ++bx)
             tma_load_5d(sbase + L::kV + vs * L::kTileBytes + bx * L::kBoxBytes, &tm_v,
@@ -327,7 +351,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
       auto wt = [&](uint32_t bar_addr, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait_lean(bar_addr, parity, ctl));
       };
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kKeys, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
       const SmemDesc dq = SmemDesc::sw128(sbase + L::kQ, 16, 1024);
       const SmemDesc dk = SmemDesc::sw128(sbase + L::kK, 16, 1024);
@@ -352,7 +376,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kNaHalf / 16; ++kk)
             umma_ts_elect(tmem + L::col_o(h, i), tmem + sb * 128 + h * kNaHalf + kk * 8,
-                          dv.at(v_off + (h * kNaHalf + kk * 16) * 128), idesc_pv,
+                          dv.at(v_off + (h * kGrpKeys + kk * 16) * 128), idesc_pv,
                           (j > 0 || kk > 0) ? 1u : 0u);
           umma_commit_elect(bar(L::bOD + h));
         }
@@ -411,9 +435,8 @@ __global__ void __launch_bounds__(kNaThreads, 1)
     const int lt = row / (BX * BY), ly = (row / BX) % BY, lx = row % BX;
     const float sl2 = p.scale_log2;
     const float2 sc2 = make_float2(sl2, sl2);
-    constexpr int kRows = kNaHalf / KX;   // (t, y) rows of a tile in this group's half
-    constexpr int kRowsChunk = 32 / KX;  // rows per 32-key chunk
-    const int r0 = grp * kRows;          // the half's first row in the tile
+    constexpr int kRows = kGrpKeys / KX;  // (t, y) rows of a tile in this group's half
+    const int r0 = grp * kRows;           // the half's first row in the tile
     bool ok = !*abort_flag;
     int g = 0;
     Brick cur;
@@ -432,10 +455,18 @@ __global__ void __launch_bounds__(kNaThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::bSF + sb), (uint32_t)(g >> 1) & 1u, ctl));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tS = tlane + sb * 128 + grp * kNaHalf;
-        float s[kNaHalf];
-        tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(&s[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+        const uint32_t tS = tlane + sb * 128 + grp * kGrpKeys;  // this half's scores
+        const uint32_t tP = tlane + sb * 128 + grp * kNaHalf;   // its P: 64 keys, 32 columns
+        float s[kGrpKeys];
+        if constexpr (kGrpKeys % 32 == 0) {
+#pragma unroll
+          for (int c = 0; c < kGrpKeys / 32; ++c)
+            tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < kGrpKeys / 8; ++c)
+            tmem_ld8(tS + c * 8, *reinterpret_cast<float(*)[8]>(&s[c * 8]));
+        }
         int kt, ky, kx;
         cur.key_origin(j, kt, ky, kx);
         const uint32_t mt = na_bits(wt0 - kt, wt0 - kt + p.win_t, KT);
@@ -474,6 +505,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
             a = fmax3(a, sr[c], sr[c + 1]);
             b = fmax3(b, sr[c + 2], sr[c + 3]);
           }
+          if constexpr (KX % 4 == 2) a = fmax3(a, sr[KX - 2], sr[KX - 1]);
           mrow = (rows_in >> r) & 1u ? fmax3(mrow, a, b) : mrow;
         }
         const float mx_t = mrow * sl2;
@@ -515,13 +547,19 @@ __global__ void __launch_bounds__(kNaThreads, 1)
 #pragma unroll
         for (int c = 0; c < kNaHalf / 32; ++c) {
           // a 32-key chunk outside every window of this warp's rows: P = 0 without the
-          // exponentials
-          const uint32_t chunk_rows = (rows_in >> (c * kRowsChunk)) & ((1u << kRowsChunk) - 1u);
+          // exponentials; P past this half's keys is 0
+          const int ra = c * 32 / KX;
+          const int rb = (c * 32 + 31 < kGrpKeys ? c * 32 + 31 : kGrpKeys - 1) / KX;
+          const uint32_t chunk_rows = rows_in & (((2u << rb) - 1u) & ~((1u << ra) - 1u));
           uint32_t pk[16];
           if (__any_sync(0xffffffffu, chunk_rows != 0)) {
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
               const int k = c * 32 + 2 * x;
+              if (k >= kGrpKeys) {
+                pk[x] = 0u;
+                continue;
+              }
               const float2 a = __ffma2_rn(make_float2(s[k], s[k + 1]), sc2, nm2[k / KX]);
               const float2 e = make_float2(ex2(a.x), ex2(a.y));
               if (x & 1)
@@ -534,7 +572,7 @@ __global__ void __launch_bounds__(kNaThreads, 1)
 #pragma unroll
             for (int x = 0; x < 16; ++x) pk[x] = 0u;
           }
-          tmem_st16(tS + c * 16, pk);
+          tmem_st16(tP + c * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();

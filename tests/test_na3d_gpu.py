@@ -2,9 +2,9 @@
 
 Same bar as the attention parity tests: max-abs error <= 2e-2 and relative L2 error
 <= 5e-3 on the bf16 output.  The grids are chosen so that the host picks each of the
-six (query brick, key tile) shape pairs (bricks 2x8x8, 1x8x16, 4x4x8; key tiles of the
-brick's own shape, 4x2x16 or 1x16x8), with ragged bricks on every axis, one and two heads,
-batch 1 and 2, head_dim 64 and 128.
+seven (query brick, key tile) shape pairs (bricks 2x8x8, 1x8x16, 4x4x8; key tiles of the
+brick's own shape, 4x2x16, 1x16x8 or the 112-key 4x2x14), with ragged bricks on every axis,
+one and two heads, batch 1 and 2, head_dim 64 and 128.
 """
 import numpy as np
 import pytest
@@ -40,7 +40,7 @@ CASES = [
     # batch, grid (T, Y, X), heads, head_dim, window   query brick (key tile) the host picks
     (1, (2, 8, 8), 1, 64, (1, 3, 3)),      # 2x8x8, a single brick
     (2, (3, 10, 13), 2, 64, (3, 5, 7)),    # 4x4x8, ragged on every axis
-    (1, (5, 12, 20), 2, 128, (3, 7, 7)),   # 2x8x8
+    (1, (5, 12, 20), 2, 128, (3, 7, 7)),   # 2x8x8 bricks over 4x2x14 key tiles (112 keys)
     (2, (1, 24, 40), 2, 64, (1, 7, 9)),    # 1x8x16 (1x16x8 key tiles), a 2-D grid
     (1, (16, 8, 8), 1, 128, (7, 3, 3)),    # 2x8x8, long time axis
     (1, (12, 6, 9), 2, 64, (5, 3, 5)),     # 2x8x8, bricks wider than the grid
@@ -48,9 +48,12 @@ CASES = [
     (1, (1, 5, 6), 1, 64, (1, 3, 5)),      # a grid smaller than one brick on every axis
     (2, (3, 10, 13), 2, 128, (3, 5, 7)),   # 4x4x8 at head_dim 128, batch 2
     (1, (9, 4, 5), 3, 128, (5, 3, 3)),     # 4x4x8, three heads, long time axis
-    (1, (2, 3, 40), 2, 64, (1, 3, 9)),     # 1x8x16, long thin grid
-    (1, (8, 12, 16), 2, 128, (3, 3, 9)),   # 2x8x8 bricks over 4x2x16 key tiles
-    (1, (6, 12, 16), 2, 64, (3, 5, 5)),    # 2x8x8 / 4x2x16 at head_dim 64
+    (1, (2, 3, 40), 2, 64, (1, 3, 9)),     # 2x8x8, long thin grid
+    (1, (8, 12, 16), 2, 128, (3, 3, 9)),   # 2x8x8 bricks over 4x2x14 key tiles
+    (1, (6, 12, 16), 2, 64, (3, 5, 5)),    # 2x8x8 / 4x2x14 at head_dim 64
+    (1, (6, 12, 32), 2, 64, (3, 5, 9)),    # 2x8x8 / 4x2x16 (x boxes of 16)
+    (2, (6, 13, 30), 2, 128, (3, 7, 7)),   # 2x8x8 / 4x2x14, ragged, batch 2
+    (1, (5, 11, 29), 2, 64, (3, 5, 7)),    # 2x8x8 / 4x2x14 at head_dim 64, ragged
     (2, (3, 9, 17), 2, 64, (3, 3, 9)),     # 4x4x8 bricks over 4x2x16 key tiles, ragged
     (1, (4, 14, 22), 1, 128, (3, 7, 7)),   # 4x4x8 / 4x2x16 at head_dim 128
 ]
@@ -104,8 +107,8 @@ def test_deterministic():
 
 @pytest.mark.parametrize("win", [(3, 7, 7), (5, 9, 9)], ids=["w3x7x7", "w5x9x9"])
 def test_decoder_grid_sampled_rows(win):
-    # the bench grid, 16 x 34 x 60 tokens (2x8x8 bricks for 3x7x7, 4x4x8 for 5x9x9, both
-    # over 4x2x16 key tiles),
+    # the bench grid, 16 x 34 x 60 tokens (2x8x8 bricks over 4x2x14 key tiles for 3x7x7, 4x4x8
+    # bricks over 4x2x16 for 5x9x9),
     # 32 heads x 128; every head of a seeded sample of tokens, including the grid's corners
     grid, h, d = (16, 34, 60), 32, 128
     n = grid[0] * grid[1] * grid[2]
