@@ -53,7 +53,7 @@ TRAFFIC = {
                    "note": "ncu_small capture (B1 8192 tokens), scaled linearly by tokens"},
     "qk_prologue": {"src": "75b060c4d34193c3", "bytes": 511.267584e6 + 446.194176e6,
                     "note": "full launch, B2 x 15360 x 32 x 128, q and k"},
-    "na3d_decoder": {"src": "9c815a5c2b547aad", "bytes": 802.395136e6 + 248.623104e6,
+    "na3d_decoder": {"src": "7986839b9164a1e4", "bytes": 802.395136e6 + 248.623104e6,
                      "note": "full launch, 16x34x60 grid, 3x7x7 window, 32x128"},
 }
 

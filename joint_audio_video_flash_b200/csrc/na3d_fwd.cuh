@@ -11,19 +11,21 @@
 //
 // Blocking: a query tile is a brick of BT x BY x BX = 128 tokens (one 5-D TMA box, rows in
 // raster order inside the brick).  The keys any of its queries can see form a box (the
-// union of their windows); it is covered by key tiles that are KT x KY x KX bricks of 128
-// keys starting at the box's corner (one 5-D TMA box each, zero fill past the grid), so a
-// query brick meets nt * ny * nx key tiles.  The key tile's shape is chosen apart from the
-// query brick's, to cover the box with as few tiles as possible (a 2 x 8 x 8 brick's box
-// for a 3 x 7 x 7 window, 4 x 14 x 14, takes seven 4 x 2 x 16 tiles but eight 2 x 8 x 8).
+// union of their windows); it is covered by key tiles that are KT x KY x KX bricks of 112
+// or 128 keys starting at the box's corner (one 5-D TMA box each, zero fill past the grid),
+// so a query brick meets nt * ny * nx key tiles.  The key tile's shape is chosen apart from
+// the query brick's, to cover the box with as few tiles and keys as possible (a 2 x 8 x 8
+// brick's box for a 3 x 7 x 7 window, 4 x 14 x 14, is exactly seven 4 x 2 x 14 tiles; it
+// takes seven 4 x 2 x 16 or eight 2 x 8 x 8 ones of 128 keys).
 // The scores of every tile are masked per element against the query row's own window:
 // a bias of 0 or -inf per key column x, and per (t, y) row of the tile a choice between the
 // row's max offset and -inf in the exponent (three bit masks, one per axis); a warp skips
 // the exponentials of each 32-key chunk that lies outside all of its rows' windows.
 //
-// Two softmax warpgroups split every key tile: group 0 takes its keys [0, 64), group 1 its
-// keys [64, 128).  Each keeps its own running max, row sum and O accumulator (two PV
-// products per tile, one per half of the keys), so the groups never wait for each other
+// Two softmax warpgroups split every key tile into halves of whole key rows: group g takes
+// keys [n g, n g + n), n = 56 or 64, and writes their P as 64 keys (zero past its n) over
+// columns [64 g, 64 g + 32) of S.  Each keeps its own running max, row sum and O accumulator
+// (two PV products per tile, one per half), so the groups never wait for each other
 // inside a brick and every SM sub-partition runs two softmax warps; the halves are merged
 // once per brick (the group-0 statistics go to group 1 through shared memory, group 1
 // writes both halves' weights, the epilogue sums the two O's with them).
@@ -44,7 +46,9 @@
 //               it with one 5-D TMA store (clipped at the grid's edges), overlapping the
 //               next brick's MMAs; the Q stage returns to the producer once the store has
 //               read it.
-// TMEM (512 columns): S0 [0,128), S1 [128,256); from 256 the O accumulators, one per group
+// TMEM (512 columns): S0 [0,128), S1 [128,256) (a 112-key tile's QK writes the first 112
+// columns; rows 112-127 of every V stage are zeroed once, since the second half's PV reads V
+// rows up to 119 with P = 0 there); from 256 the O accumulators, one per group
 // (head_dim 128), or one per group and brick parity (head_dim 64: 4 x 64 columns).
 // Registers (setmaxnreg): producer/MMA warpgroup 88, softmax 168 (each group), epilogue 88.
 #pragma once
