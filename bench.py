@@ -1176,34 +1176,13 @@ def run_prologue(args):
 
 
 # (query brick, key tile) pairs the library is built for, as t x y x x
-NA_SHAPES = (((2, 8, 8), (2, 8, 8)), ((2, 8, 8), (4, 2, 16)), ((1, 8, 16), (1, 8, 16)),
-             ((1, 8, 16), (1, 16, 8)), ((4, 4, 8), (4, 4, 8)), ((4, 4, 8), (4, 2, 16)),
-             ((2, 8, 8), (4, 2, 14)))
-
-
 def na_key_tiles(grid, window, with_shape=False):
-    """Key tiles the neighbourhood kernel multiplies per (batch, head), for the shape pair the
-    library picks: the fewest tiles, then the fewest keys in all tiles (counting only; no
-    attention math).  With with_shape, also the query brick and key tile shapes."""
-    def start(i, k, n):
-        return min(max(i - k // 2, 0), n - k)
-
-    def axis(n, blk, kblk, k):
-        tot = 0
-        for a0 in range(0, n, blk):
-            a1 = min(a0 + blk, n)
-            r0, r1 = start(a0, k, n), start(a1 - 1, k, n) + k
-            tot += -(-(r1 - r0) // kblk)
-        return tot
-
-    best = None
-    for qb, kb in NA_SHAPES:
-        tiles = (axis(grid[0], qb[0], kb[0], window[0]) * axis(grid[1], qb[1], kb[1], window[1])
-                 * axis(grid[2], qb[2], kb[2], window[2]))
-        key = (tiles, tiles * kb[0] * kb[1] * kb[2])
-        if best is None or key < best[0]:
-            best = (key, tiles, qb, kb)
-    return best[1:] if with_shape else best[1]
+    """Key tiles the neighbourhood kernel multiplies per (batch, head), from the library's own
+    plan (``ltxattn_na3d_plan``, host only).  With with_shape, also the query brick and key
+    tile shapes."""
+    from joint_audio_video_flash_b200 import ltxattn
+    brick, tile, tiles = ltxattn.na3d_plan(grid, window)
+    return (tiles, brick, tile) if with_shape else tiles
 
 
 def na_issued_flops(grid, window, b, heads, d):

@@ -268,6 +268,20 @@ LTXATTN_API int ltxattn_na3d_forward(const void* q, const void* k, const void* v
                                      float scale, ltxattn_stream_t stream);
 
 /*
+ * The blocking ltxattn_na3d_forward uses for a grid and window, on the host only (no
+ * device, no ltxattn_create): of the query brick / key tile shape pairs the kernel is built
+ * for, the one whose bricks meet the fewest key tiles in all, then the fewest keys.
+ *   shape   host int[6]: the query brick (t, y, x), then the key tile (t, y, x); the brick
+ *           holds 128 tokens, the key tile 112 or 128 keys
+ *   tiles   host: key tiles per (batch, head), i.e. the 128-query x (key tile) products
+ *           the tensor cores multiply per (batch, head)
+ * Same grid and window rules as ltxattn_na3d_forward (LTXATTN_ERR_INVALID_ARG otherwise,
+ * and also for null pointers); LTXATTN_OK with both outputs written.
+ */
+LTXATTN_API int ltxattn_na3d_plan(int grid_t, int grid_y, int grid_x, int window_t, int window_y,
+                                  int window_x, int* shape, long long* tiles);
+
+/*
  * Attention over one key range, left unnormalised across ranges: the building block of
  * context-parallel attention, where each rank holds a shard of the keys and values and the
  * ranks exchange per-range results in fp32 with their softmax statistics ("feat(ltx2):

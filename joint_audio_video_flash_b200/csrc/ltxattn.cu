@@ -66,6 +66,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
     "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope", "ltxattn_na3d_forward",
     "ltxattn_forward_partial", "ltxattn_combine", "ltxattn_forward_grouped",
+    "ltxattn_na3d_plan",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -422,6 +423,34 @@ long long na_tiles_total(const NaShape& b, int t, int y, int x, int kt, int ky, 
     return sum;
   };
   return axis(t, b.bt, b.kt, kt) * axis(y, b.by, b.ky, ky) * axis(x, b.bx, b.kx, kx);
+}
+
+// The shape pair (an index into kNaShapes) with the fewest key tiles over all bricks, then
+// the fewest keys; its tile count per (batch, head) in *tiles when tiles is not null.
+int na_pick(int t, int y, int x, int wt, int wy, int wx, long long* tiles) {
+  int best = 0;
+  long long best_keys = -1, best_tiles = -1;
+  for (int i = 0; i < kNumNaShapes; ++i) {
+    const NaShape& s = kNaShapes[i];
+    const long long n = na_tiles_total(s, t, y, x, wt, wy, wx);
+    const long long keys = n * (s.kt * s.ky * s.kx);
+    if (best_tiles < 0 || n < best_tiles || (n == best_tiles && keys < best_keys)) {
+      best_keys = keys;
+      best_tiles = n;
+      best = i;
+    }
+  }
+  if (tiles) *tiles = best_tiles;
+  return best;
+}
+
+// Grid and window rules of the neighbourhood entry points.
+bool na_grid_ok(int grid_t, int grid_y, int grid_x, int window_t, int window_y, int window_x) {
+  if (grid_t < 1 || grid_y < 1 || grid_x < 1) return false;
+  const int grid_dims[3] = {grid_t, grid_y, grid_x}, win[3] = {window_t, window_y, window_x};
+  for (int a = 0; a < 3; ++a)
+    if (win[a] < 1 || win[a] % 2 == 0 || win[a] > grid_dims[a]) return false;
+  return true;
 }
 
 // BSHD bf16 tensor over a T x Y x X grid, [batch, T*Y*X, heads, head_dim], seen as a 5-D
@@ -904,11 +933,9 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
                          int window_t, int window_y, int window_x, float scale,
                          ltxattn_stream_t stream_) {
   if (!q || !k || !v || !out) return LTXATTN_ERR_INVALID_ARG;
-  if (batch < 1 || heads < 1 || grid_t < 1 || grid_y < 1 || grid_x < 1)
+  if (batch < 1 || heads < 1 ||
+      !na_grid_ok(grid_t, grid_y, grid_x, window_t, window_y, window_x))
     return LTXATTN_ERR_INVALID_ARG;
-  const int grid_dims[3] = {grid_t, grid_y, grid_x}, win[3] = {window_t, window_y, window_x};
-  for (int a = 0; a < 3; ++a)
-    if (win[a] < 1 || win[a] % 2 == 0 || win[a] > grid_dims[a]) return LTXATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.0f)) return LTXATTN_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return LTXATTN_ERR_UNSUPPORTED;
   const long long tokens = (long long)grid_t * grid_y * grid_x;
@@ -925,18 +952,7 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
   Context* c = current_context(&st);
   if (!c) return st;
 
-  int best = 0;
-  long long best_keys = -1, best_tiles = -1;
-  for (int i = 0; i < kNumNaShapes; ++i) {
-    const NaShape& s = kNaShapes[i];
-    const long long t = na_tiles_total(s, grid_t, grid_y, grid_x, window_t, window_y, window_x);
-    const long long keys = t * (s.kt * s.ky * s.kx);
-    if (best_tiles < 0 || t < best_tiles || (t == best_tiles && keys < best_keys)) {
-      best_keys = keys;
-      best_tiles = t;
-      best = i;
-    }
-  }
+  const int best = na_pick(grid_t, grid_y, grid_x, window_t, window_y, window_x, nullptr);
   const NaShape& sh = kNaShapes[best];
   ltx::Na3dParams p{};
   p.batch = batch;
@@ -969,6 +985,17 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
       head_dim == 64 ? launch_na<64>(best, tq, tk, tv, to, p, c->num_sms, stream, shapes)
                      : launch_na<128>(best, tq, tk, tv, to, p, c->num_sms, stream, shapes);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
+int ltxattn_na3d_plan(int grid_t, int grid_y, int grid_x, int window_t, int window_y,
+                      int window_x, int* shape, long long* tiles) {
+  if (!shape || !tiles || !na_grid_ok(grid_t, grid_y, grid_x, window_t, window_y, window_x))
+    return LTXATTN_ERR_INVALID_ARG;
+  const NaShape& s = kNaShapes[na_pick(grid_t, grid_y, grid_x, window_t, window_y, window_x,
+                                       tiles)];
+  const int v[6] = {s.bt, s.by, s.bx, s.kt, s.ky, s.kx};
+  for (int i = 0; i < 6; ++i) shape[i] = v[i];
+  return LTXATTN_OK;
 }
 
 int ltxattn_forward_partial(const void* q, const void* k, const void* v, float* o_part,

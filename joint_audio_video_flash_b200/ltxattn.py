@@ -55,6 +55,7 @@ def load() -> ctypes.CDLL:
             lib.ltxattn_qk_norm_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci,
                                                  cf, vp]
             lib.ltxattn_na3d_forward.argtypes = [vp, vp, vp, vp] + [ci] * 9 + [cf, vp]
+            lib.ltxattn_na3d_plan.argtypes = [ci] * 6 + [vp, vp]
             lib.ltxattn_forward_partial.argtypes = [vp, vp, vp, vp, vp] + [ci] * 6 + [cf, vp]
             lib.ltxattn_combine.argtypes = [vp, vp, vp] + [ci] * 5 + [vp]
             lib.ltxattn_forward_grouped.argtypes = [vp, ci, vp]
@@ -291,6 +292,18 @@ def na3d_forward(q, k, v, grid, window, out=None, *, scale: float | None = None,
         ctypes.c_void_p(_stream_handle(stream)))
     _check(st, "ltxattn_na3d_forward")
     return out
+
+
+def na3d_plan(grid, window):
+    """The blocking ``ltxattn_na3d_forward`` uses (``ltxattn_na3d_plan``, host only): the
+    query brick (t, y, x), the key tile (t, y, x) and the key tiles per (batch, head)."""
+    shape = (ctypes.c_int * 6)()
+    tiles = ctypes.c_longlong()
+    st = load().ltxattn_na3d_plan(*(int(x) for x in grid), *(int(x) for x in window),
+                                  ctypes.cast(shape, ctypes.c_void_p),
+                                  ctypes.cast(ctypes.pointer(tiles), ctypes.c_void_p))
+    _check(st, "ltxattn_na3d_plan")
+    return tuple(shape[:3]), tuple(shape[3:]), int(tiles.value)
 
 
 def rows_pad(q_len: int) -> int:
