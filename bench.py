@@ -59,21 +59,24 @@ TRAFFIC = {
 
 
 def kernel_label(c, num_sms: int = 148, grouped: bool = False) -> str:
-    """Name of the kernel the library's host dispatch picks for a call (report label only)."""
-    qt = -(-c.q_len // 128)
+    """Name of the kernel the library's host dispatch picks for a call (report label only),
+    from the library's own plan (``ltxattn_forward_plan``, host only)."""
+    from joint_audio_video_flash_b200 import ltxattn
     kt = -(-c.kv_valid_len // 128)
-    if c.head_dim == 64 and kt == 1 and (grouped or c.batch * c.heads * qt > num_sms):
-        return "ltx_attn_fwd_a2v (persistent, per-unit K/V" + (
-            ", grouped launch)" if grouped else ")")
-    if kt <= 2 and c.batch * c.heads * qt > num_sms:
-        return f"ltx_attn_fwd_skv<{c.head_dim}, {kt}> (persistent, K/V resident)"
-    if c.head_dim == 64 and kt > 2 and qt <= 1:
-        return "ltx_attn_fwd<64, 1 S buffer> (two CTAs per SM)"
-    if c.head_dim == 128 and qt >= 8 and (kt < 4 or c.batch * c.heads * ((qt + 1) // 2) >= num_sms):
-        return "ltx_attn_fwd_pair (CTA pairs, cta_group::2, four query tiles per pair)"
-    if qt >= 2:
-        return f"ltx_attn_fwd_pp<{c.head_dim}> (two 128-row query tiles per CTA)"
-    return f"ltx_attn_fwd<{c.head_dim}>"
+    if grouped and c.head_dim == 64 and kt == 1:
+        return "ltx_attn_fwd_a2v (persistent, per-unit K/V, grouped launch)"
+    kernel, _ = ltxattn.forward_plan(c.q_len, c.kv_len, c.kv_valid_len, c.batch, c.heads,
+                                     c.head_dim, 0, num_sms)
+    d = c.head_dim
+    return {
+        ltxattn.KERNEL_A2V: "ltx_attn_fwd_a2v (persistent, per-unit K/V)",
+        ltxattn.KERNEL_SHORT_KV:
+            f"ltx_attn_fwd_skv<{d}, {2 if d == 64 else kt}> (persistent, K/V resident)",
+        ltxattn.KERNEL_ONE_TILE_DUAL: "ltx_attn_fwd<64, 1 S buffer> (two CTAs per SM)",
+        ltxattn.KERNEL_PAIR: "ltx_attn_fwd_pair (CTA pairs, cta_group::2, four query tiles per pair)",
+        ltxattn.KERNEL_TWO_TILES: f"ltx_attn_fwd_pp<{d}> (two 128-row query tiles per CTA)",
+        ltxattn.KERNEL_ONE_TILE: f"ltx_attn_fwd<{d}>",
+    }[kernel]
 
 
 GROUP_MAX = 4  # calls per launch of the grouped kernel

@@ -281,6 +281,28 @@ LTXATTN_API int ltxattn_na3d_forward(const void* q, const void* k, const void* v
 LTXATTN_API int ltxattn_na3d_plan(int grid_t, int grid_y, int grid_x, int window_t, int window_y,
                                   int window_x, int* shape, long long* tiles);
 
+/* The attention kernels ltxattn_forward chooses between (ltxattn_forward_plan). */
+typedef enum ltxattn_kernel {
+  LTXATTN_KERNEL_ONE_TILE = 0,       /* one 128-row query tile per CTA, S double-buffered */
+  LTXATTN_KERNEL_TWO_TILES = 1,      /* two query tiles per CTA, softmax ping-pong */
+  LTXATTN_KERNEL_ONE_TILE_DUAL = 2,  /* head_dim 64, one query tile: two CTAs per SM */
+  LTXATTN_KERNEL_SHORT_KV = 3,       /* persistent, every valid key in one or two tiles */
+  LTXATTN_KERNEL_A2V = 4,            /* persistent, head_dim 64, one key tile (groupable) */
+  LTXATTN_KERNEL_PAIR = 5            /* head_dim 128, CTA pairs (cta_group::2) */
+} ltxattn_kernel;
+
+/*
+ * Which kernel ltxattn_forward (and ltxattn_forward_ex with `num_splits`) runs for a call of
+ * these sizes on a GPU with `num_sms` SMs, and into how many key-range parts it splits the
+ * keys (1 = no split; more = fp32 partials and a merge kernel), on the host only: no device,
+ * no ltxattn_create.  Sizes follow ltxattn_forward's rules (INVALID_ARG / UNSUPPORTED as
+ * there); num_splits >= 0; num_sms >= 1; kernel and parts are host pointers, written on
+ * LTXATTN_OK.
+ */
+LTXATTN_API int ltxattn_forward_plan(int q_len, int kv_len, int kv_valid_len, int batch,
+                                     int heads, int head_dim, int num_splits, int num_sms,
+                                     int* kernel, int* parts);
+
 /*
  * Attention over one key range, left unnormalised across ranges: the building block of
  * context-parallel attention, where each rank holds a shard of the keys and values and the

@@ -66,7 +66,7 @@ const char* const kEntryPoints[] = {
     "ltxattn_selftest_wait_timeout", "ltxattn_num_entry_points", "ltxattn_entry_point_name",
     "ltxattn_forward_split_noalloc", "ltxattn_qk_norm_rope", "ltxattn_na3d_forward",
     "ltxattn_forward_partial", "ltxattn_combine", "ltxattn_forward_grouped",
-    "ltxattn_na3d_plan",
+    "ltxattn_na3d_plan", "ltxattn_forward_plan",
 };
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -75,9 +75,9 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 // All checks that need no CUDA call, in the order the header documents.
-int validate(const void* q, const void* k, const void* v, void* out, int q_len, int kv_len,
-             int kv_valid_len, int batch, int heads, int head_dim, float scale) {
-  if (!q || !k || !v || !out) return LTXATTN_ERR_INVALID_ARG;
+// The size rules of an attention call (no pointers).
+int validate_sizes(int q_len, int kv_len, int kv_valid_len, int batch, int heads, int head_dim,
+                   float scale) {
   if (q_len < 1 || kv_len < 1 || batch < 1 || heads < 1) return LTXATTN_ERR_INVALID_ARG;
   if (kv_valid_len < 1 || kv_valid_len > kv_len) return LTXATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.0f)) return LTXATTN_ERR_INVALID_ARG;
@@ -85,6 +85,14 @@ int validate(const void* q, const void* k, const void* v, void* out, int q_len, 
   if (q_len > LTXATTN_MAX_LEN || kv_len > LTXATTN_MAX_LEN || heads > LTXATTN_MAX_HEADS ||
       batch > LTXATTN_MAX_BATCH)
     return LTXATTN_ERR_UNSUPPORTED;
+  return LTXATTN_OK;
+}
+
+int validate(const void* q, const void* k, const void* v, void* out, int q_len, int kv_len,
+             int kv_valid_len, int batch, int heads, int head_dim, float scale) {
+  if (!q || !k || !v || !out) return LTXATTN_ERR_INVALID_ARG;
+  const int st = validate_sizes(q_len, kv_len, kv_valid_len, batch, heads, head_dim, scale);
+  if (st != LTXATTN_OK) return st;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                         reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out);
   if (mis & 15u) return LTXATTN_ERR_MISALIGNED;
@@ -539,6 +547,15 @@ cudaError_t launch_pair(const CUtensorMap& tq, const CUtensorMap& tk_half, const
   return cudaGetLastError();
 }
 
+// The attention kernel a planned call runs (the values of ltxattn_kernel).
+int kernel_family(const FwdParams& p, int head_dim, bool dual, int num_sms) {
+  if (use_pair(p, head_dim, num_sms)) return LTXATTN_KERNEL_PAIR;
+  if (use_short_kv(p, num_sms))
+    return a2v_eligible(p, head_dim) ? LTXATTN_KERNEL_A2V : LTXATTN_KERNEL_SHORT_KV;
+  if (dual) return LTXATTN_KERNEL_ONE_TILE_DUAL;
+  return p.n_q_tiles >= 2 ? LTXATTN_KERNEL_TWO_TILES : LTXATTN_KERNEL_ONE_TILE;
+}
+
 // Launches the planned kernel (and, with key-range parts, the merge into `out`).  `tk_half`
 // is the key map with 64-row boxes, used by the pair kernel.
 cudaError_t launch_planned(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -546,12 +563,13 @@ cudaError_t launch_planned(const CUtensorMap& tq, const CUtensorMap& tk, const C
                            int num_sms, void* out, cudaStream_t stream,
                            const CUtensorMap* tk_half = nullptr) {
   const bool split = p.num_splits > 1;
+  const int family = kernel_family(p, head_dim, dual, num_sms);
   cudaError_t e;
-  if (tk_half && use_pair(p, head_dim, num_sms)) {
+  if (tk_half && family == LTXATTN_KERNEL_PAIR) {
     return launch_pair(tq, *tk_half, tv, to, p, stream);
-  } else if (use_short_kv(p, num_sms)) {
+  } else if (family == LTXATTN_KERNEL_A2V || family == LTXATTN_KERNEL_SHORT_KV) {
     return launch_skv(tq, tk, tv, to, p, head_dim, num_sms, stream);
-  } else if (dual) {
+  } else if (family == LTXATTN_KERNEL_ONE_TILE_DUAL) {
     e = split ? launch_fwd<64, true, 1>(tq, tk, tv, to, p, stream)
               : launch_fwd<64, false, 1>(tq, tk, tv, to, p, stream);
   } else if (head_dim == 64) {
@@ -985,6 +1003,26 @@ int ltxattn_na3d_forward(const void* q, const void* k, const void* v, void* out,
       head_dim == 64 ? launch_na<64>(best, tq, tk, tv, to, p, c->num_sms, stream, shapes)
                      : launch_na<128>(best, tq, tk, tv, to, p, c->num_sms, stream, shapes);
   return e == cudaSuccess ? LTXATTN_OK : LTXATTN_ERR_CUDA;
+}
+
+int ltxattn_forward_plan(int q_len, int kv_len, int kv_valid_len, int batch, int heads,
+                         int head_dim, int num_splits, int num_sms, int* kernel, int* parts) {
+  if (!kernel || !parts || num_splits < 0 || num_sms < 1) return LTXATTN_ERR_INVALID_ARG;
+  const int st = validate_sizes(q_len, kv_len, kv_valid_len, batch, heads, head_dim, 1.0f);
+  if (st != LTXATTN_OK) return st;
+  FwdParams p{};
+  p.q_len = q_len;
+  p.kv_len = kv_len;
+  p.kv_valid = kv_valid_len;
+  p.heads = heads;
+  p.batch = batch;
+  p.n_q_tiles = (q_len + ltx::kBlockM - 1) / ltx::kBlockM;
+  p.n_kv_tiles = (kv_valid_len + ltx::kBlockN - 1) / ltx::kBlockN;
+  const bool dual = plan_kernel(p, head_dim, num_splits, num_sms, 0);
+  if ((long long)batch * p.num_splits > 65535) return LTXATTN_ERR_UNSUPPORTED;
+  *kernel = kernel_family(p, head_dim, dual, num_sms);
+  *parts = p.num_splits;
+  return LTXATTN_OK;
 }
 
 int ltxattn_na3d_plan(int grid_t, int grid_y, int grid_x, int window_t, int window_y,

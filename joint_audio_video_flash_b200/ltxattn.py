@@ -56,6 +56,7 @@ def load() -> ctypes.CDLL:
                                                  cf, vp]
             lib.ltxattn_na3d_forward.argtypes = [vp, vp, vp, vp] + [ci] * 9 + [cf, vp]
             lib.ltxattn_na3d_plan.argtypes = [ci] * 6 + [vp, vp]
+            lib.ltxattn_forward_plan.argtypes = [ci] * 8 + [vp, vp]
             lib.ltxattn_forward_partial.argtypes = [vp, vp, vp, vp, vp] + [ci] * 6 + [cf, vp]
             lib.ltxattn_combine.argtypes = [vp, vp, vp] + [ci] * 5 + [vp]
             lib.ltxattn_forward_grouped.argtypes = [vp, ci, vp]
@@ -292,6 +293,25 @@ def na3d_forward(q, k, v, grid, window, out=None, *, scale: float | None = None,
         ctypes.c_void_p(_stream_handle(stream)))
     _check(st, "ltxattn_na3d_forward")
     return out
+
+
+# ltxattn_kernel values
+KERNEL_ONE_TILE, KERNEL_TWO_TILES, KERNEL_ONE_TILE_DUAL = 0, 1, 2
+KERNEL_SHORT_KV, KERNEL_A2V, KERNEL_PAIR = 3, 4, 5
+
+
+def forward_plan(q_len: int, kv_len: int, kv_valid_len: int, batch: int, heads: int,
+                 head_dim: int, num_splits: int = 0, num_sms: int = 148):
+    """The kernel ``ltxattn_forward`` runs for these sizes and its key-range parts
+    (``ltxattn_forward_plan``, host only): (one of the KERNEL_* values, parts)."""
+    kernel = ctypes.c_int()
+    parts = ctypes.c_int()
+    st = load().ltxattn_forward_plan(int(q_len), int(kv_len), int(kv_valid_len), int(batch),
+                                     int(heads), int(head_dim), int(num_splits), int(num_sms),
+                                     ctypes.cast(ctypes.pointer(kernel), ctypes.c_void_p),
+                                     ctypes.cast(ctypes.pointer(parts), ctypes.c_void_p))
+    _check(st, "ltxattn_forward_plan")
+    return kernel.value, parts.value
 
 
 def na3d_plan(grid, window):
